@@ -1,0 +1,164 @@
+"""B200-native canvas denoise-sampling stage for uniform-state block diffusion.
+
+Thin Python binding over the C ABI of ``include/dg.h`` (``libdg.so``).  The
+functions here only marshal torch tensors into pointers; every step of the path
+runs in the library's sm_100a kernels.  There is no CPU or PyTorch fallback: if
+the library is missing, importing a function that needs it raises.
+"""
+
+import ctypes
+
+import torch
+
+from . import _abi
+from ._abi import DgError, DgParams, check, lib
+
+__all__ = ["DgError", "DgParams", "params", "workspace_size", "plan", "temperature", "dg_canvas_init",
+           "dg_denoise_step", "dg_stop_check", "dg_stub_hidden", "last_launch_count", "Workspace",
+           "decode_batch", "decode_block_ar"]
+
+
+def params(n_canvas, vocab, hidden, **overrides):
+    """dg_params with the pages' defaults (48 steps, T 0.8->0.4, bound 0.1, stop 0.005, stability 2)."""
+    p = DgParams()
+    lib().dg_params_default(ctypes.byref(p), int(n_canvas), int(vocab), int(hidden))
+    for k, v in overrides.items():
+        if not hasattr(p, k):
+            raise KeyError(k)
+        setattr(p, k, v)
+    return p
+
+
+def workspace_size(p):
+    n = lib().dg_workspace_size(ctypes.byref(p))
+    if n == 0:
+        raise DgError("dg_workspace_size", _abi.DG_EINVAL, "invalid or unsupported params")
+    return n
+
+
+def plan(p):
+    g, ng, sl = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    check("dg_plan", lib().dg_plan(ctypes.byref(p), ctypes.byref(g), ctypes.byref(ng), ctypes.byref(sl)))
+    return {"group": g.value, "n_groups": ng.value, "slice": sl.value}
+
+
+def temperature(p, step):
+    return float(lib().dg_temperature(ctypes.byref(p), int(step)))
+
+
+def last_launch_count():
+    return int(lib().dg_last_launch_count())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+class Workspace:
+    """Device workspace for one dg_params (caller-owned memory, as the ABI requires)."""
+
+    def __init__(self, p, device="cuda"):
+        self.params = p
+        self.nbytes = workspace_size(p)
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+
+    @property
+    def ptr(self):
+        return ctypes.c_void_p(self.buf.data_ptr())
+
+
+def dg_canvas_init(p, seeds, tokens, ws, stream=None):
+    check("dg_canvas_init", lib().dg_canvas_init(ctypes.byref(p), _ptr(seeds), _ptr(tokens), ws.ptr,
+                                                 ws.nbytes, _stream(stream)))
+
+
+def dg_denoise_step(p, step, h, W, E, seeds, tokens, entropy, argmax, accept, lse, selfcond, ws, stream=None):
+    check("dg_denoise_step", lib().dg_denoise_step(
+        ctypes.byref(p), int(step), _ptr(h), _ptr(W), _ptr(E), _ptr(seeds), _ptr(tokens), _ptr(entropy),
+        _ptr(argmax), _ptr(accept), _ptr(lse), _ptr(selfcond), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def dg_stop_check(p, ws, stream=None, want_stable=False):
+    """Synchronises the stream; returns (stop_flags list, stable list or None, n_stopped)."""
+    C = p.n_canvas
+    flags = (ctypes.c_int32 * C)()
+    stable = (ctypes.c_int32 * C)() if want_stable else None
+    n = ctypes.c_int()
+    check("dg_stop_check", lib().dg_stop_check(ctypes.byref(p), ws.ptr, ws.nbytes, flags,
+                                               stable if stable is not None else None, ctypes.byref(n),
+                                               _stream(stream)))
+    return list(flags), (list(stable) if stable is not None else None), n.value
+
+
+def dg_stub_hidden(p, step, gain, noise, seeds, E, tokens, h, ws, stream=None):
+    check("dg_stub_hidden", lib().dg_stub_hidden(ctypes.byref(p), int(step), float(gain), float(noise),
+                                                 _ptr(seeds), _ptr(E), _ptr(tokens), _ptr(h), ws.ptr, ws.nbytes,
+                                                 _stream(stream)))
+
+
+class StepBuffers:
+    """Per-step outputs for N positions (device tensors)."""
+
+    def __init__(self, p, device="cuda", selfcond=True):
+        N, d = p.n_canvas * p.canvas_len, p.hidden
+        self.tokens = torch.empty(N, dtype=torch.int32, device=device)
+        self.entropy = torch.empty(N, dtype=torch.float32, device=device)
+        self.argmax = torch.empty(N, dtype=torch.int32, device=device)
+        self.accept = torch.empty(N, dtype=torch.uint8, device=device)
+        self.lse = torch.empty(N, dtype=torch.float32, device=device)
+        self.selfcond = torch.empty((N, d), dtype=torch.float32, device=device) if selfcond else None
+        self.h = torch.empty((N, d), dtype=torch.bfloat16, device=device)
+
+
+def decode_batch(p, W, E, seeds, gain=1.0, noise=0.1, hidden_fn=None, ws=None, bufs=None, on_step=None):
+    """Denoise C independent canvases together until each stops or reaches max_steps.
+
+    hidden_fn(tokens, step) -> h fills the denoiser's hidden states; by default the
+    benchmark stub (dg_stub_hidden) stands in for the network.  Stopped canvases
+    cost nothing in later steps.  Returns (committed [C, 256] int32, stop_step list).
+    """
+    ws = ws or Workspace(p, W.device)
+    bufs = bufs or StepBuffers(p, W.device)
+    dg_canvas_init(p, seeds, bufs.tokens, ws)
+    C = p.n_canvas
+    stop_step = [p.max_steps] * C
+    for s in range(1, p.max_steps + 1):
+        if hidden_fn is None:
+            dg_stub_hidden(p, s, gain, noise, seeds, E, bufs.tokens, bufs.h, ws)
+        else:
+            bufs.h.copy_(hidden_fn(bufs.tokens, s))
+        dg_denoise_step(p, s, bufs.h, W, E, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept, bufs.lse,
+                        bufs.selfcond, ws)
+        if on_step is not None:
+            on_step(s, bufs)
+        flags, _, n_stopped = dg_stop_check(p, ws)
+        for c in range(C):
+            if flags[c] and stop_step[c] == p.max_steps and s < p.max_steps:
+                stop_step[c] = s
+        if n_stopped == C:
+            break
+    return bufs.argmax.view(C, p.canvas_len).clone(), stop_step
+
+
+def decode_block_ar(p1, W, E, n_blocks, seed0=0, gain=1.0, noise=0.1):
+    """Block-autoregressive decoding: n_blocks canvases of 256 tokens one after another.
+
+    p1 describes one canvas (n_canvas = 1); canvas b uses seed seed0 + b.  The
+    committed block of each canvas is appended to the output.  Returns (tokens
+    [n_blocks * 256] int32, per-block stop steps).
+    """
+    ws = Workspace(p1, W.device)
+    bufs = StepBuffers(p1, W.device)
+    out, steps = [], []
+    for b in range(n_blocks):
+        seeds = torch.tensor([seed0 + b], dtype=torch.int64, device=W.device)
+        committed, st = decode_batch(p1, W, E, seeds, gain, noise, ws=ws, bufs=bufs)
+        out.append(committed.view(-1))
+        steps.append(st[0])
+    return torch.cat(out), steps

@@ -1,0 +1,357 @@
+// C ABI of the denoise-sampling stage: argument checks, planning, workspace
+// layout, TMA descriptor encoding and the launch sequence of one step.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/dg.h"
+#include "dg_common.cuh"
+#include "dg_fused.h"
+
+using namespace dg;
+
+namespace {
+
+constexpr int kFusedSmem = 4 * 48 * 1024 + 1024 + 4 * kMaxCanvas;
+thread_local int g_last_launches = 0;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+int device_sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    return sms;
+}
+
+bool params_ok(const dg_params* p) {
+    if (!p) return false;
+    if (p->n_canvas < 1 || p->n_canvas > kMaxCanvas) return false;
+    if (p->canvas_len != kCanvas) return false;
+    if (p->vocab < kBV || p->vocab % kBV != 0) return false;
+    if (p->hidden < 64 || p->hidden % 64 != 0) return false;
+    if (p->max_steps < 1) return false;
+    if (!(p->t_start > 0.f) || !(p->t_end > 0.f)) return false;
+    if (p->stability < 0) return false;
+    return true;
+}
+
+// Returns DG_OK and fills `pl`, or the reason the shape is not handled.
+dg_status make_plan(const dg_params* p, int sms, Plan* pl) {
+    if (!params_ok(p)) return DG_EINVAL;
+    int slice = 0;
+    if (p->group > 0) {
+        if (p->hidden % p->group != 0) return DG_EUNSUPPORTED;
+        slice = p->hidden / p->group;
+        if (slice % 64 != 0 || slice > kMaxSlice) return DG_EUNSUPPORTED;
+    } else {
+        for (int s = kMaxSlice; s >= 64; s -= 64)
+            if (p->hidden % s == 0) {
+                slice = s;
+                break;
+            }
+    }
+    const int G = p->hidden / slice;
+    if (sms < G) return DG_EUNSUPPORTED;
+    Plan q{};
+    q.C = p->n_canvas;
+    q.N = p->n_canvas * kCanvas;
+    q.V = p->vocab;
+    q.d = p->hidden;
+    q.group = G;
+    q.slice = slice;
+    q.n_groups = sms / G;
+    q.steps_per_tile = (p->vocab + G * kBV - 1) / (G * kBV);
+    const long long U = 2LL * q.C * q.steps_per_tile;
+    const long long per_group = (U + q.n_groups - 1) / q.n_groups;
+    q.max_seg = static_cast<int>((per_group + q.steps_per_tile - 1) / q.steps_per_tile) + 1;
+    q.n_slots = q.n_groups * q.max_seg;
+    *pl = q;
+    return DG_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+               uint32_t box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <class T>
+T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+}  // namespace
+
+extern "C" {
+
+void dg_params_default(dg_params* p, int n_canvas, int vocab, int hidden) {
+    if (!p) return;
+    std::memset(p, 0, sizeof(*p));
+    p->n_canvas = n_canvas;
+    p->canvas_len = kCanvas;
+    p->vocab = vocab;
+    p->hidden = hidden;
+    p->max_steps = 48;
+    p->t_start = 0.8f;
+    p->t_end = 0.4f;
+    p->eb_bound = 0.1f;
+    p->stop_thresh = 0.005f;
+    p->stability = 2;
+    p->tied = 1;
+    p->group = 0;
+}
+
+float dg_temperature(const dg_params* p, int step) {
+    if (!p) return NAN;
+    double t = p->t_start;
+    if (p->max_steps > 1)
+        t = static_cast<double>(p->t_start) +
+            (static_cast<double>(p->t_end) - static_cast<double>(p->t_start)) * (step - 1) / (p->max_steps - 1);
+    return static_cast<float>(t);
+}
+
+const char* dg_status_string(dg_status s) {
+    switch (s) {
+        case DG_OK: return "ok";
+        case DG_EINVAL: return "invalid argument";
+        case DG_ECUDA: return "CUDA error";
+        case DG_EUNSUPPORTED: return "unsupported shape";
+        case DG_ETIMEOUT: return "in-kernel wait timed out";
+        case DG_ENOMEM: return "workspace too small";
+    }
+    return "unknown status";
+}
+
+int dg_last_launch_count(void) { return g_last_launches; }
+
+dg_status dg_plan(const dg_params* p, int* group, int* n_groups, int* slice_cols) {
+    const int sms = device_sm_count();
+    if (sms <= 0) return DG_ECUDA;
+    Plan pl;
+    dg_status st = make_plan(p, sms, &pl);
+    if (st != DG_OK) return st;
+    if (group) *group = pl.group;
+    if (n_groups) *n_groups = pl.n_groups;
+    if (slice_cols) *slice_cols = pl.slice;
+    return DG_OK;
+}
+
+size_t dg_workspace_size(const dg_params* p) {
+    const int sms = device_sm_count();
+    if (sms <= 0) return 0;
+    Plan pl;
+    if (make_plan(p, sms, &pl) != DG_OK) return 0;
+    return make_layout(pl).total;
+}
+
+dg_status dg_canvas_init(const dg_params* p, const uint64_t* seeds_dev, int32_t* tokens_dev, void* workspace_dev,
+                         size_t workspace_bytes, void* stream) {
+    g_last_launches = 0;
+    const int sms = device_sm_count();
+    if (sms <= 0) return DG_ECUDA;
+    Plan pl;
+    dg_status st = make_plan(p, sms, &pl);
+    if (st != DG_OK) return st;
+    if (!seeds_dev || !tokens_dev || !workspace_dev) return DG_EINVAL;
+    const Layout L = make_layout(pl);
+    if (workspace_bytes < L.total) return DG_ENOMEM;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int threads = 256;
+    const int blocks = (pl.N + threads - 1) / threads;
+    dg_init_kernel<<<blocks, threads, 0, s>>>(seeds_dev, tokens_dev, at<int32_t>(workspace_dev, L.prev_argmax),
+                                              at<int32_t>(workspace_dev, L.stable), at<int32_t>(workspace_dev, L.stop),
+                                              at<int32_t>(workspace_dev, L.err), at<uint32_t>(workspace_dev, L.counters),
+                                              pl.n_groups * 128, pl.C, pl.V);
+    if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
+    g_last_launches = 1;
+    return DG_OK;
+}
+
+dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const void* W_dev, const void* E_dev,
+                          const uint64_t* seeds_dev, int32_t* tokens_dev, float* entropy_dev, int32_t* argmax_dev,
+                          uint8_t* accept_dev, float* lse_dev, float* selfcond_dev, void* workspace_dev,
+                          size_t workspace_bytes, void* stream) {
+    g_last_launches = 0;
+    const int sms = device_sm_count();
+    if (sms <= 0) return DG_ECUDA;
+    Plan pl;
+    dg_status st = make_plan(p, sms, &pl);
+    if (st != DG_OK) return st;
+    if (step < 1 || step > p->max_steps) return DG_EINVAL;
+    if (!h_dev || !W_dev || !E_dev || !seeds_dev || !tokens_dev || !entropy_dev || !argmax_dev || !accept_dev ||
+        !workspace_dev)
+        return DG_EINVAL;
+    if (!aligned16(h_dev) || !aligned16(W_dev) || !aligned16(E_dev) || (selfcond_dev && !aligned16(selfcond_dev)))
+        return DG_EINVAL;
+    const Layout L = make_layout(pl);
+    if (workspace_bytes < L.total) return DG_ENOMEM;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(dg_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem);
+    });
+    if (attr_err != cudaSuccess) return DG_ECUDA;
+
+    const float T = dg_temperature(p, step);
+    FusedArgs fa;
+    std::memset(&fa, 0, sizeof(fa));
+    const uint64_t prow_total = static_cast<uint64_t>(pl.n_groups) * 2 * pl.group * kTileM;
+    if (!encode_2d(&fa.map_h, h_dev, pl.N, pl.d, 64, kTileM) || !encode_2d(&fa.map_w, W_dev, pl.V, pl.d, 64, kBV) ||
+        !encode_2d(&fa.map_e, E_dev, pl.V, pl.d, 64, kVChunk) ||
+        !encode_2d(&fa.map_p, at<void>(workspace_dev, L.pbuf), prow_total, kBV, 64, kTileM))
+        return DG_ECUDA;
+    int32_t* stop = at<int32_t>(workspace_dev, L.stop);
+    fa.stop = stop;
+    fa.counters = at<uint32_t>(workspace_dev, L.counters);
+    fa.rowmax = at<float>(workspace_dev, L.rowmax);
+    fa.pbuf = at<__nv_bfloat16>(workspace_dev, L.pbuf);
+    fa.stats = at<float4>(workspace_dev, L.stats);
+    fa.stat_idx = at<int32_t>(workspace_dev, L.stat_idx);
+    fa.opart = at<float>(workspace_dev, L.opart);
+    fa.err = at<int>(workspace_dev, L.err);
+    fa.C = pl.C;
+    fa.V = pl.V;
+    fa.d = pl.d;
+    fa.G = pl.group;
+    fa.slice = pl.slice;
+    fa.n_groups = pl.n_groups;
+    fa.steps_per_tile = pl.steps_per_tile;
+    fa.max_seg = pl.max_seg;
+    fa.scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
+
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(pl.n_groups * pl.group);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kFusedSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, dg_fused_kernel, fa) != cudaSuccess) return DG_ECUDA;
+
+    CombineArgs ca;
+    ca.stop = stop;
+    ca.counters = fa.counters;
+    ca.stats = fa.stats;
+    ca.stat_idx = fa.stat_idx;
+    ca.opart = fa.opart;
+    ca.entropy = entropy_dev;
+    ca.argmax = argmax_dev;
+    ca.lse = lse_dev;
+    ca.selfcond = selfcond_dev;
+    ca.C = pl.C;
+    ca.d = pl.d;
+    ca.G = pl.group;
+    ca.n_groups = pl.n_groups;
+    ca.steps_per_tile = pl.steps_per_tile;
+    ca.max_seg = pl.max_seg;
+    dg_combine_kernel<<<pl.N, 256, 0, s>>>(ca);
+    if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
+
+    dg_accept_kernel<<<(pl.N + 255) / 256, 256, 0, s>>>(entropy_dev, argmax_dev, seeds_dev, stop, tokens_dev,
+                                                         accept_dev, p->eb_bound, step, pl.N, pl.V);
+    if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
+
+    dg_stop_kernel<<<pl.C, kCanvas, 0, s>>>(entropy_dev, argmax_dev, at<int32_t>(workspace_dev, L.prev_argmax),
+                                            at<int32_t>(workspace_dev, L.stable), stop, p->stop_thresh, p->stability,
+                                            step);
+    if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
+    g_last_launches = 4;
+    return DG_OK;
+}
+
+dg_status dg_stop_check(const dg_params* p, void* workspace_dev, size_t workspace_bytes, int32_t* stop_flags_host,
+                        int32_t* stable_host, int* n_stopped_host, void* stream) {
+    const int sms = device_sm_count();
+    if (sms <= 0) return DG_ECUDA;
+    Plan pl;
+    dg_status st = make_plan(p, sms, &pl);
+    if (st != DG_OK) return st;
+    if (!workspace_dev) return DG_EINVAL;
+    const Layout L = make_layout(pl);
+    if (workspace_bytes < L.total) return DG_ENOMEM;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t err_word = 0;
+    if (cudaMemcpyAsync(&err_word, at<int32_t>(workspace_dev, L.err), sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
+        cudaSuccess)
+        return DG_ECUDA;
+    int32_t flags_local[kMaxCanvas];
+    int32_t* flags = stop_flags_host ? stop_flags_host : flags_local;
+    if (cudaMemcpyAsync(flags, at<int32_t>(workspace_dev, L.stop), sizeof(int32_t) * pl.C, cudaMemcpyDeviceToHost,
+                        s) != cudaSuccess)
+        return DG_ECUDA;
+    if (stable_host && cudaMemcpyAsync(stable_host, at<int32_t>(workspace_dev, L.stable), sizeof(int32_t) * pl.C,
+                                       cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return DG_ECUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return DG_ECUDA;
+    if (n_stopped_host) {
+        int n = 0;
+        for (int c = 0; c < pl.C; ++c) n += flags[c] != 0;
+        *n_stopped_host = n;
+    }
+    if (err_word != 0) return DG_ETIMEOUT;
+    return DG_OK;
+}
+
+dg_status dg_stub_hidden(const dg_params* p, int step, float gain, float noise, const uint64_t* seeds_dev,
+                         const void* E_dev, const int32_t* tokens_dev, void* h_dev, void* workspace_dev,
+                         size_t workspace_bytes, void* stream) {
+    g_last_launches = 0;
+    const int sms = device_sm_count();
+    if (sms <= 0) return DG_ECUDA;
+    Plan pl;
+    dg_status st = make_plan(p, sms, &pl);
+    if (st != DG_OK) return st;
+    if (step < 1 || step > p->max_steps) return DG_EINVAL;
+    if (!seeds_dev || !E_dev || !tokens_dev || !h_dev || !workspace_dev) return DG_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(E_dev) & 7u) || (reinterpret_cast<uintptr_t>(h_dev) & 7u)) return DG_EINVAL;
+    const Layout L = make_layout(pl);
+    if (workspace_bytes < L.total) return DG_ENOMEM;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const float a_s = static_cast<float>(static_cast<double>(step) / p->max_steps);
+    const long long total = static_cast<long long>(pl.N) * (pl.d / 4);
+    long long blocks = (total + 255) / 256;
+    if (blocks > static_cast<long long>(sms) * 16) blocks = static_cast<long long>(sms) * 16;
+    dg_stub_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(
+        seeds_dev, static_cast<const __nv_bfloat16*>(E_dev), tokens_dev, at<int32_t>(workspace_dev, L.stop),
+        static_cast<__nv_bfloat16*>(h_dev), a_s, gain, noise, step, pl.d, pl.V, pl.N);
+    if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
+    g_last_launches = 1;
+    return DG_OK;
+}
+
+}  // extern "C"

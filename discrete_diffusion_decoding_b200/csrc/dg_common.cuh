@@ -1,0 +1,113 @@
+// Shared definitions of the CUDA library: the Philox generator, the workspace
+// layout and the schedule that maps (position tile, vocabulary block) work onto
+// groups of CTAs of the fused kernel.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/dg.h"
+
+namespace dg {
+
+constexpr int kCanvas = 256;      // positions per canvas
+constexpr int kTileM = 128;       // positions per tile (UMMA M)
+constexpr int kBV = 256;          // vocabulary rows per logits tile (UMMA N)
+constexpr int kKChunk = 64;       // hidden columns per pipeline stage of the logits GEMM
+constexpr int kVChunk = 64;       // vocabulary rows per pipeline stage of the self-conditioning GEMM
+constexpr int kMaxSlice = 256;    // widest self-conditioning column slice one CTA keeps in TMEM
+constexpr int kMaxCanvas = 1024;  // canvases per call (the fused kernel keeps the active list in shared memory)
+constexpr int kThreads = 256;     // threads of the fused kernel
+constexpr float kLazyRescale = 8.0f;  // log2 units the shared reference may lag the running max
+
+// ------------------------------------------------------------------ Philox4x32-10
+// Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3" (SC'11):
+// ten rounds; per round the two 32x32->64 products of counter words 0 and 2 with
+// the multipliers, the high halves xored with the other words and the key; the key
+// advances by the Weyl increments between rounds.
+__host__ __device__ inline void philox4x32_10(uint32_t c[4], uint32_t k0, uint32_t k1) {
+    for (int r = 0; r < 10; ++r) {
+        if (r) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c[0];
+        const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c[2];
+        const uint32_t n0 = static_cast<uint32_t>(p1 >> 32) ^ c[1] ^ k0;
+        const uint32_t n1 = static_cast<uint32_t>(p1);
+        const uint32_t n2 = static_cast<uint32_t>(p0 >> 32) ^ c[3] ^ k1;
+        const uint32_t n3 = static_cast<uint32_t>(p0);
+        c[0] = n0;
+        c[1] = n1;
+        c[2] = n2;
+        c[3] = n3;
+    }
+}
+
+// floor(word0 * V / 2^32) for counter (i, s, c, tag) under the canvas seed.
+__host__ __device__ inline int32_t philox_token(uint64_t seed, uint32_t i, uint32_t s, uint32_t c, uint32_t tag,
+                                                uint32_t vocab) {
+    uint32_t ctr[4] = {i, s, c, tag};
+    philox4x32_10(ctr, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
+    return static_cast<int32_t>((static_cast<uint64_t>(ctr[0]) * vocab) >> 32);
+}
+
+enum : uint32_t { kTagInit = 0, kTagRenoise = 1, kTagStubTarget = 2, kTagStubNoise = 3 };
+
+// ------------------------------------------------------------------ plan and layout
+struct Plan {
+    int C, N, V, d;
+    int group;        // G: CTAs sharing one logits tile stream, each owning d/G columns
+    int slice;        // d / G
+    int n_groups;     // groups resident at once (grid = n_groups * G CTAs)
+    int steps_per_tile;  // vocabulary blocks of G * kBV rows per position tile
+    int max_seg;      // partial slots per group
+    int n_slots;      // n_groups * max_seg
+};
+
+struct Layout {
+    size_t prev_argmax, stable, stop, err;        // per-canvas state
+    size_t counters;                              // [n_groups][4] uint32, 128 B apart
+    size_t rowmax;                                // [n_groups][2][G][128] float
+    size_t pbuf;                                  // [n_groups][2][G][128][kBV] bf16
+    size_t stats;                                 // [n_slots][G][128] float4 {m, l, u, best}
+    size_t stat_idx;                              // [n_slots][G][128] int32
+    size_t opart;                                 // [n_slots][128][d] float
+    size_t total;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline Layout make_layout(const Plan& pl) {
+    Layout L{};
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o = align_up(o + bytes, 256);
+        return at;
+    };
+    L.prev_argmax = take(sizeof(int32_t) * pl.N);
+    L.stable = take(sizeof(int32_t) * pl.C);
+    L.stop = take(sizeof(int32_t) * pl.C);
+    L.err = take(sizeof(int32_t) * 4);
+    L.counters = take(static_cast<size_t>(128) * 4 * pl.n_groups);
+    L.rowmax = take(sizeof(float) * pl.n_groups * 2 * pl.group * kTileM);
+    L.pbuf = take(static_cast<size_t>(2) * pl.n_groups * 2 * pl.group * kTileM * kBV);
+    L.stats = take(sizeof(float) * 4 * pl.n_slots * pl.group * kTileM);
+    L.stat_idx = take(sizeof(int32_t) * pl.n_slots * pl.group * kTileM);
+    L.opart = take(sizeof(float) * static_cast<size_t>(pl.n_slots) * kTileM * pl.d);
+    L.total = o;
+    return L;
+}
+
+// Units of work: (position tile, vocabulary block) pairs numbered tile-major;
+// group g owns the contiguous range [unit_begin(g), unit_begin(g+1)).
+__host__ __device__ inline long long unit_begin(int g, long long U, int n_groups) {
+    return (static_cast<long long>(g) * U) / n_groups;
+}
+
+// Offsets of the four per-group counters (uint32 words).
+enum : int { kCntRowmax = 0, kCntP = 1, kCntUsed = 2 };
+__host__ __device__ inline size_t counter_word(int g, int which) { return static_cast<size_t>(g) * 128 + which * 32; }
+
+}  // namespace dg

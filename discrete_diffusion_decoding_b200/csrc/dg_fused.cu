@@ -1,0 +1,624 @@
+// Fused denoise-sampling pass (logits, online softmax statistics, entropy,
+// argmax and self-conditioning) and the split-vocabulary combine.
+//
+// Method (juhoplayground "DiffusionGemma", inference mechanism: logits for
+// every canvas position, temperature sharpening, self-conditioning with the
+// probability-weighted token embedding; marrrang deep dive, reverse-diffusion
+// steps 3-5 and the entropy criteria):
+//   z = h W^T / T;  p = softmax(z);  H = LSE - sum p z;  a = argmax z;  sc = p E.
+//
+// Work decomposition (sm_100a, one CTA per SM, persistent, cooperative launch):
+//  * A position tile is 128 canvas positions (UMMA M = 128).
+//  * A group of G CTAs streams the vocabulary in blocks of G x 256 rows.  In a
+//    block, CTA r computes the 256-wide logits tile of vocabulary sub-tile r over
+//    the full hidden width (TMA -> SMEM -> tcgen05.mma -> TMEM), and owns columns
+//    [r*d/G, (r+1)*d/G) of the self-conditioning accumulator O (fp32, in TMEM).
+//  * The G CTAs agree on a per-row reference maximum for the block (row maxima
+//    exchanged through L2 with release/acquire counters), so every CTA turns its
+//    logits tile into P = 2^(z*log2e - m_ref) in bf16 against the same reference,
+//    publishes P to an L2-resident scratch tile, and accumulates
+//    O[:, slice] += P_q E[q-rows, slice] for all G tiles q of the block (second
+//    tcgen05 GEMM, E as an MN-major operand).  The reference only moves when the
+//    running maximum exceeds it by 8 (log2 units), and then O is rescaled in TMEM.
+//  * Each CTA keeps exact per-row partial statistics of its own tiles relative
+//    to the shared reference: l = sum e, u = sum e (z - m_ref), and the best raw
+//    logit with its smallest vocabulary index.
+//  * A group's contiguous range of (position tile, block) units is split at tile
+//    boundaries into segments; each segment ends with O and the statistics
+//    written as a partial, merged by dg_combine_kernel.
+//
+// Roles inside a CTA (256 threads): warp 0 issues TMA loads into a 4-stage ring
+// of 48 KB stages; warp 1 allocates TMEM and issues UMMAs; warps 4-7 (one TMEM
+// lane quarter each, thread = position row) do the softmax, publish P and run
+// the epilogue.  Every wait is bounded (see dg_sm100.cuh).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "dg_common.cuh"
+#include "dg_fused.h"
+#include "dg_sm100.cuh"
+
+namespace dg {
+
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kStageBytes = 48 * 1024;     // S stage: h 16 KB + W 32 KB; O stage: P 16 KB + E 32 KB
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemS = 0;             // logits tile columns [0, 256)
+constexpr uint32_t kTmemO = 256;           // self-conditioning slice columns [256, 256 + slice)
+constexpr int kSoftmaxWarp0 = 4;
+
+// error codes recorded in the workspace error word
+enum : int {
+    kErrProducerEmpty = 101, kErrProducerP = 102, kErrProducerDrain = 103,
+    kErrMmaFull = 201, kErrMmaSFree = 202, kErrMmaOReady = 203, kErrMmaDrain = 204,
+    kErrSmaxSFull = 301, kErrSmaxRowmax = 302, kErrSmaxUsed = 303, kErrSmaxODone = 304,
+};
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Bounded poll until *ctr >= target (wrap-safe comparison).
+__device__ bool wait_counter(const uint32_t* ctr, uint32_t target, volatile int* abort, int* err, int code) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        if (static_cast<int32_t>(ld_acquire_u32(ctr) - target) >= 0) return true;
+        if (*abort) return false;
+        if ((it & 15u) == 0) {
+            const uint64_t now = global_ns();
+            if (it == 0) {
+                t0 = now;
+            } else if (now - t0 > DG_WAIT_LIMIT_NS) {
+                atomicCAS(err, 0, code);
+                *abort = 1;
+                return false;
+            }
+        }
+        __nanosleep(32);
+    }
+}
+
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    uint32_t a[16], b[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        a[i] = r[i];
+        b[i] = r[16 + i];
+    }
+    tmem_st16(taddr, a);
+    tmem_st16(taddr + 16, b);
+}
+
+// The contiguous unit range of one group, split into segments at tile boundaries.
+struct Schedule {
+    long long u0, u1;
+    int T;
+    int pt0;
+    int nseg;
+    __device__ void init(int g, int n_groups, int n_pt, int steps_per_tile) {
+        T = steps_per_tile;
+        const long long U = static_cast<long long>(n_pt) * T;
+        u0 = unit_begin(g, U, n_groups);
+        u1 = unit_begin(g + 1, U, n_groups);
+        if (u1 > u0) {
+            pt0 = static_cast<int>(u0 / T);
+            nseg = static_cast<int>((u1 - 1) / T) - pt0 + 1;
+        } else {
+            pt0 = 0;
+            nseg = 0;
+        }
+    }
+    __device__ void seg(int j, int& pt, int& tb, int& te) const {
+        pt = pt0 + j;
+        const long long base = static_cast<long long>(pt) * T;
+        const long long lo = u0 > base ? u0 : base;
+        const long long hi = u1 < base + T ? u1 : base + T;
+        tb = static_cast<int>(lo - base);
+        te = static_cast<int>(hi - base);
+    }
+};
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_constant__ FusedArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    int* active = reinterpret_cast<int*>(ring + kStages * kStageBytes);
+
+    __shared__ uint64_t full_bar[kStages], empty_bar[kStages];
+    __shared__ uint64_t s_full, s_free, o_ready, o_done, drain_bar;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    __shared__ int n_active_s;
+    __shared__ int rescale_any;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int G = a.G;
+    const int g = blockIdx.x / G;
+    const int r = blockIdx.x % G;
+    const int d0 = r * a.slice;
+
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full_bar[i], 1);
+            mbar_init(&empty_bar[i], 1);
+        }
+        mbar_init(&s_full, 1);
+        mbar_init(&s_free, 1);
+        mbar_init(&o_ready, 1);
+        mbar_init(&o_done, 1);
+        mbar_init(&drain_bar, 1);
+        fence_mbar_init_cluster();
+        abort_flag = 0;
+        rescale_any = 0;
+    }
+    if (warp == 2) {
+        // active canvases in increasing order
+        int base = 0;
+        for (int c0 = 0; c0 < a.C; c0 += 32) {
+            const int c = c0 + lane;
+            const bool act = c < a.C && a.stop[c] == 0;
+            const uint32_t m = __ballot_sync(0xffffffffu, act);
+            if (act) active[base + __popc(m & ((1u << lane) - 1u))] = c;
+            base += __popc(m);
+        }
+        if (lane == 0) n_active_s = base;
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem = tmem_base;
+    Schedule sch;
+    sch.init(g, a.n_groups, 2 * n_active_s, a.steps_per_tile);
+    auto sub_valid = [&](int t, int q) { return static_cast<long long>(t * G + q) * kBV < a.V; };
+    auto vocab0 = [&](int t, int q) { return (t * G + q) * kBV; };
+    auto row0_of = [&](int pt) { return active[pt >> 1] * kCanvas + (pt & 1) * kTileM; };
+
+    uint32_t* cnt_rowmax = a.counters + counter_word(g, kCntRowmax);
+    uint32_t* cnt_p = a.counters + counter_word(g, kCntP);
+    uint32_t* cnt_used = a.counters + counter_word(g, kCntUsed);
+    const int n_ech = a.slice / 64;                 // E boxes per O stage
+    const uint32_t o_stage_bytes = 16384u + static_cast<uint32_t>(n_ech) * 8192u;
+
+    if (warp == 0) {
+        // ===================================================== TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&a.map_h);
+            tma_prefetch_desc(&a.map_w);
+            tma_prefetch_desc(&a.map_e);
+            tma_prefetch_desc(&a.map_p);
+            uint32_t it = 0;
+            bool ok = true;
+            auto acquire = [&](int& slot) -> bool {
+                slot = static_cast<int>(it % kStages);
+                if (it >= kStages &&
+                    !mbar_wait(&empty_bar[slot], ((it / kStages) - 1) & 1, &abort_flag, a.err, kErrProducerEmpty))
+                    return false;
+                ++it;
+                return true;
+            };
+            auto emit_o = [&](int k, int t) -> bool {
+                if (!wait_counter(cnt_p, static_cast<uint32_t>(G * (k + 1)), &abort_flag, a.err, kErrProducerP))
+                    return false;
+                fence_async_global();
+                for (int q = 0; q < G; ++q) {
+                    if (!sub_valid(t, q)) continue;
+                    const int prow = ((g * 2 + (k & 1)) * G + q) * kTileM;
+                    for (int c4 = 0; c4 < kBV / kVChunk; ++c4) {
+                        int slot;
+                        if (!acquire(slot)) return false;
+                        uint8_t* st = ring + slot * kStageBytes;
+                        mbar_arrive_expect_tx(&full_bar[slot], o_stage_bytes);
+                        tma_load_2d(st, &a.map_p, &full_bar[slot], c4 * kVChunk, prow);
+                        for (int j = 0; j < n_ech; ++j)
+                            tma_load_2d(st + 16384 + j * 8192, &a.map_e, &full_bar[slot], d0 + j * 64,
+                                        vocab0(t, q) + c4 * kVChunk);
+                    }
+                }
+                return true;
+            };
+            int k = 0;
+            for (int j = 0; j < sch.nseg && ok; ++j) {
+                int pt, tb, te;
+                sch.seg(j, pt, tb, te);
+                const int row0 = row0_of(pt);
+                for (int t = tb; t < te && ok; ++t, ++k) {
+                    if (sub_valid(t, r)) {
+                        const int v0 = vocab0(t, r);
+                        for (int kc = 0; kc < a.d / kKChunk; ++kc) {
+                            int slot;
+                            if (!acquire(slot)) { ok = false; break; }
+                            uint8_t* st = ring + slot * kStageBytes;
+                            mbar_arrive_expect_tx(&full_bar[slot], 16384u + 32768u);
+                            tma_load_2d(st, &a.map_h, &full_bar[slot], kc * kKChunk, row0);
+                            tma_load_2d(st + 16384, &a.map_w, &full_bar[slot], kc * kKChunk, v0);
+                        }
+                    }
+                    if (ok && t > tb) ok = emit_o(k - 1, t - 1);
+                }
+                if (ok) ok = emit_o(k - 1, te - 1);
+            }
+            // drain: every issued load must have landed before the CTA may exit
+            for (uint32_t u = (it > kStages ? it - kStages : 0); u < it; ++u) {
+                const int slot = static_cast<int>(u % kStages);
+                uint64_t t0 = global_ns();
+                while (!mbar_try_wait(smem_u32(&full_bar[slot]), (u / kStages) & 1)) {
+                    if (global_ns() - t0 > DG_WAIT_LIMIT_NS) {
+                        atomicCAS(a.err, 0, kErrProducerDrain);
+                        break;
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ===================================================== UMMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_s = idesc_bf16_f32(kTileM, kBV, false, false);
+            const uint32_t idesc_o = idesc_bf16_f32(kTileM, a.slice, false, true);
+            uint32_t it = 0;
+            bool ok = true;
+            auto consume = [&](int& slot) -> bool {
+                slot = static_cast<int>(it % kStages);
+                if (!mbar_wait(&full_bar[slot], (it / kStages) & 1, &abort_flag, a.err, kErrMmaFull)) return false;
+                ++it;
+                tc_fence_after();
+                return true;
+            };
+            // seg_first: block t is the first of its segment, so O starts from zero
+            auto do_o = [&](int k, int t, bool seg_first) -> bool {
+                if (!mbar_wait(&o_ready, k & 1, &abort_flag, a.err, kErrMmaOReady)) return false;
+                tc_fence_after();
+                bool first = seg_first;
+                for (int q = 0; q < G; ++q) {
+                    if (!sub_valid(t, q)) continue;
+                    for (int c4 = 0; c4 < kBV / kVChunk; ++c4) {
+                        int slot;
+                        if (!consume(slot)) return false;
+                        const uint32_t st = smem_u32(ring + slot * kStageBytes);
+#pragma unroll
+                        for (int kk = 0; kk < kVChunk / 16; ++kk) {
+                            const uint64_t ad = smem_desc(st + kk * 32, 16, 1024, kSwizzle128B);
+                            const uint64_t bd = smem_desc(st + 16384 + kk * 2048, 8192, 1024, kSwizzle128B);
+                            umma_ss(tmem + kTmemO, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
+                        }
+                        first = false;
+                        umma_commit(&empty_bar[slot]);
+                    }
+                }
+                // every P tile of block k has landed in this CTA's shared memory
+                red_release_add(cnt_used, 1u);
+                umma_commit(&o_done);
+                return true;
+            };
+            int k = 0;
+            for (int j = 0; j < sch.nseg && ok; ++j) {
+                int pt, tb, te;
+                sch.seg(j, pt, tb, te);
+                for (int t = tb; t < te && ok; ++t, ++k) {
+                    if (k > 0 && !mbar_wait(&s_free, (k - 1) & 1, &abort_flag, a.err, kErrMmaSFree)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (sub_valid(t, r)) {
+                        for (int kc = 0; kc < a.d / kKChunk; ++kc) {
+                            int slot;
+                            if (!consume(slot)) { ok = false; break; }
+                            const uint32_t st = smem_u32(ring + slot * kStageBytes);
+#pragma unroll
+                            for (int kk = 0; kk < kKChunk / 16; ++kk) {
+                                const uint64_t ad = smem_desc(st + kk * 32, 16, 1024, kSwizzle128B);
+                                const uint64_t bd = smem_desc(st + 16384 + kk * 32, 16, 1024, kSwizzle128B);
+                                umma_ss(tmem + kTmemS, ad, bd, idesc_s, (kc | kk) != 0 ? 1u : 0u);
+                            }
+                            umma_commit(&empty_bar[slot]);
+                        }
+                        if (!ok) break;
+                        umma_commit(&s_full);
+                    } else {
+                        mbar_arrive(&s_full);
+                    }
+                    if (t > tb) ok = do_o(k - 1, t - 1, t - 1 == tb);
+                }
+                if (ok) ok = do_o(k - 1, te - 1, te - 1 == tb);
+            }
+            // drain: all issued UMMAs complete before TMEM is released
+            umma_commit(&drain_bar);
+            uint64_t t0 = global_ns();
+            while (!mbar_try_wait(smem_u32(&drain_bar), 0)) {
+                if (global_ns() - t0 > DG_WAIT_LIMIT_NS) {
+                    atomicCAS(a.err, 0, kErrMmaDrain);
+                    break;
+                }
+            }
+        }
+    } else if (warp >= kSoftmaxWarp0) {
+        // ===================================================== softmax / epilogue
+        const int row = (warp - kSoftmaxWarp0) * 32 + lane;
+        const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const bool leader = (tid == kSoftmaxWarp0 * 32);
+        const float c2 = a.scale_log2;
+        bool ok = true;
+        int k = 0;
+        // Every bounded wait below is followed by a softmax-warp barrier and a
+        // check of the shared abort flag, so the 128 threads always leave
+        // together and never strand each other at a barrier.
+        for (int j = 0; j < sch.nseg && ok; ++j) {
+            int pt, tb, te;
+            sch.seg(j, pt, tb, te);
+            float m_ref = -INFINITY, l = 0.f, u = 0.f, best = -INFINITY;
+            int best_idx = -1;
+            for (int t = tb; t < te; ++t, ++k) {
+                const bool valid = sub_valid(t, r);
+                mbar_wait(&s_full, k & 1, &abort_flag, a.err, kErrSmaxSFull);
+                softmax_bar();
+                if (abort_flag) { ok = false; break; }
+                tc_fence_after();
+                // --- pass 1: row maximum of the raw logits tile
+                float smax = -INFINITY;
+                if (valid) {
+#pragma unroll 1
+                    for (int c0 = 0; c0 < kBV; c0 += 32) {
+                        uint32_t v[32];
+                        tmem_ld32(tmem + kTmemS + lane_addr + c0, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) smax = fmaxf(smax, __uint_as_float(v[i]));
+                    }
+                }
+                float* rm = a.rowmax + static_cast<size_t>((g * 2 + (k & 1)) * G) * kTileM;
+                rm[r * kTileM + row] = smax * c2;
+                __threadfence();
+                softmax_bar();
+                if (leader) {
+                    red_release_add(cnt_rowmax, 1u);
+                    bool w = wait_counter(cnt_rowmax, static_cast<uint32_t>(G * (k + 1)), &abort_flag, a.err,
+                                          kErrSmaxRowmax);
+                    // P buffer (k & 1) was last read for block k-2
+                    if (w && k >= 2)
+                        wait_counter(cnt_used, static_cast<uint32_t>(G * (k - 1)), &abort_flag, a.err, kErrSmaxUsed);
+                }
+                softmax_bar();
+                if (abort_flag) { ok = false; break; }
+                float M = -INFINITY;
+                for (int q = 0; q < G; ++q) M = fmaxf(M, __ldcg(rm + q * kTileM + row));
+                // --- lazy shared reference (the same decision in all G CTAs of the group)
+                float alpha = 1.f;
+                if (m_ref == -INFINITY || M > m_ref + kLazyRescale) {
+                    if (m_ref != -INFINITY) {
+                        alpha = exp2f(m_ref - M);
+                        u = alpha * (u + (m_ref - M) * l);
+                        l = alpha * l;
+                    }
+                    m_ref = M;
+                }
+                // --- pass 2: probabilities, statistics, argmax, P tile
+                if (valid) {
+                    __nv_bfloat16* prow =
+                        a.pbuf + (static_cast<size_t>((g * 2 + (k & 1)) * G + r) * kTileM + row) * kBV;
+                    const int v0 = vocab0(t, r);
+#pragma unroll 1
+                    for (int c0 = 0; c0 < kBV; c0 += 32) {
+                        uint32_t v[32];
+                        tmem_ld32(tmem + kTmemS + lane_addr + c0, v);
+                        tmem_wait_ld();
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            const float s0 = __uint_as_float(v[i]), s1 = __uint_as_float(v[i + 1]);
+                            if (s0 > best) { best = s0; best_idx = v0 + c0 + i; }
+                            if (s1 > best) { best = s1; best_idx = v0 + c0 + i + 1; }
+                            const float y0 = fmaf(s0, c2, -m_ref), y1 = fmaf(s1, c2, -m_ref);
+                            const float e0 = exp2f(y0), e1 = exp2f(y1);
+                            l += e0 + e1;
+                            u = fmaf(e0, y0, fmaf(e1, y1, u));
+                            pk[i / 2] = pack_bf16(e0, e1);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(prow + c0);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                }
+                tc_fence_before();
+                fence_async_global();
+                __threadfence();
+                if (alpha != 1.f && t > tb) rescale_any = 1;
+                softmax_bar();
+                const bool resc = rescale_any != 0;
+                if (leader) {
+                    mbar_arrive(&s_free);
+                    red_release_add(cnt_p, 1u);
+                }
+                // --- O of block k-1 must be complete before block k may accumulate (and be rescaled)
+                if (t > tb) {
+                    mbar_wait(&o_done, (k - 1) & 1, &abort_flag, a.err, kErrSmaxODone);
+                    softmax_bar();
+                    if (abort_flag) { ok = false; break; }
+                    tc_fence_after();
+                    if (resc) {
+#pragma unroll 1
+                        for (int c0 = 0; c0 < a.slice; c0 += 32) {
+                            uint32_t v[32];
+                            tmem_ld32(tmem + kTmemO + lane_addr + c0, v);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+                            tmem_st32(tmem + kTmemO + lane_addr + c0, v);
+                        }
+                        tmem_wait_st();
+                    }
+                    tc_fence_before();
+                }
+                softmax_bar();
+                if (leader) {
+                    rescale_any = 0;
+                    mbar_arrive(&o_ready);
+                }
+            }
+            if (!ok) break;
+            // --- segment epilogue: O slice and statistics become a partial
+            mbar_wait(&o_done, (k - 1) & 1, &abort_flag, a.err, kErrSmaxODone);
+            softmax_bar();
+            if (abort_flag) { ok = false; break; }
+            tc_fence_after();
+            const int slot = g * a.max_seg + j;
+            float* orow = a.opart + (static_cast<size_t>(slot) * kTileM + row) * a.d + d0;
+#pragma unroll 1
+            for (int c0 = 0; c0 < a.slice; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(tmem + kTmemO + lane_addr + c0, v);
+                tmem_wait_ld();
+                float4* dst = reinterpret_cast<float4*>(orow + c0);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                         __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            }
+            const size_t si = (static_cast<size_t>(slot) * G + r) * kTileM + row;
+            a.stats[si] = make_float4(m_ref, l, u, best);
+            a.stat_idx[si] = best_idx;
+            tc_fence_before();
+            softmax_bar();
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// Split-vocabulary combine: one CTA per active position.  Merges the partial
+// statistics of every (segment, rank) covering the position's tile:
+//   M = max m_s;  L = sum_s 2^(m_s-M) sum_r l;  U = sum_s 2^(m_s-M) (sum_r u + (m_s-M) sum_r l)
+//   H = ln L - ln2 * U / L;  LSE = ln2 * (M + log2 L);  argmax = best raw logit, smallest index;
+//   sc = sum_s 2^(m_s-M) O_s / L.
+// Block 0 also clears the fused kernel's group counters for its next launch.
+__global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
+    __shared__ float sh_w[64];
+    __shared__ int sh_slot[64];
+    __shared__ int n_slots_s;
+    __shared__ float sh_L;
+    __shared__ int sh_active_rank;
+    __shared__ int sh_skip;
+
+    const int n = blockIdx.x;               // position row in [0, N)
+    const int c = n / kCanvas;
+    const int tid = threadIdx.x;
+    if (blockIdx.x == 0) {
+        for (int i = tid; i < a.n_groups * 128; i += blockDim.x) a.counters[i] = 0u;
+    }
+    if (tid == 0) {
+        sh_skip = a.stop[c] != 0;
+        // rank of canvas c among the active canvases
+        int rank = 0;
+        for (int q = 0; q < c; ++q) rank += a.stop[q] == 0;
+        sh_active_rank = rank;
+    }
+    __syncthreads();
+    if (sh_skip) return;
+    int n_active = 0;
+    for (int q = 0; q < a.C; ++q) n_active += a.stop[q] == 0;   // same in every thread
+    const int pt = 2 * sh_active_rank + ((n % kCanvas) >= kTileM ? 1 : 0);
+    const int row = n % kTileM;
+    const int T = a.steps_per_tile;
+    const long long U = static_cast<long long>(2 * n_active) * T;
+
+    if (tid < 32) {
+        // warp 0: merge statistics over (slot, rank) entries
+        const long long lo = static_cast<long long>(pt) * T, hi = lo + T;
+        float M = -INFINITY;
+        int ns = 0;
+        if (tid == 0) {
+            for (int gg = 0; gg < a.n_groups; ++gg) {
+                const long long u0 = unit_begin(gg, U, a.n_groups), u1 = unit_begin(gg + 1, U, a.n_groups);
+                if (u1 <= u0 || u1 <= lo || u0 >= hi) continue;
+                const int slot = gg * a.max_seg + (pt - static_cast<int>(u0 / T));
+                if (ns < 64) sh_slot[ns++] = slot;
+            }
+            n_slots_s = ns;
+        }
+        __syncwarp();
+        ns = n_slots_s;
+        for (int s = 0; s < ns; ++s) M = fmaxf(M, a.stats[(static_cast<size_t>(sh_slot[s]) * a.G) * kTileM + row].x);
+        float L = 0.f, Uu = 0.f, best = -INFINITY;
+        int bidx = 0x7fffffff;
+        for (int e = tid; e < ns * a.G; e += 32) {
+            const int s = e / a.G, rr = e % a.G;
+            const size_t si = (static_cast<size_t>(sh_slot[s]) * a.G + rr) * kTileM + row;
+            const float4 st = a.stats[si];
+            const int idx = a.stat_idx[si];
+            const float w = exp2f(st.x - M);
+            L += w * st.y;
+            Uu += w * (st.z + (st.x - M) * st.y);
+            if (idx >= 0 && (st.w > best || (st.w == best && idx < bidx))) {
+                best = st.w;
+                bidx = idx;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) {
+            L += __shfl_xor_sync(0xffffffffu, L, off);
+            Uu += __shfl_xor_sync(0xffffffffu, Uu, off);
+            const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
+            if (ob > best || (ob == best && oi < bidx)) {
+                best = ob;
+                bidx = oi;
+            }
+        }
+        if (tid == 0) {
+            const float ln2 = 0.69314718055994531f;
+            const float H = logf(L) - ln2 * (Uu / L);
+            a.entropy[n] = H;
+            a.argmax[n] = bidx;
+            if (a.lse) a.lse[n] = ln2 * (M + log2f(L));
+            sh_L = L;
+        }
+        for (int s = tid; s < ns; s += 32) sh_w[s] = exp2f(a.stats[(static_cast<size_t>(sh_slot[s]) * a.G) * kTileM + row].x - M);
+    }
+    __syncthreads();
+    if (a.selfcond == nullptr) return;
+    const int ns = n_slots_s;
+    const float invL = 1.f / sh_L;
+    for (int col = tid * 4; col < a.d; col += blockDim.x * 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < ns; ++s) {
+            const float4 o = *reinterpret_cast<const float4*>(a.opart + (static_cast<size_t>(sh_slot[s]) * kTileM + row) * a.d + col);
+            const float w = sh_w[s];
+            acc.x = fmaf(w, o.x, acc.x);
+            acc.y = fmaf(w, o.y, acc.y);
+            acc.z = fmaf(w, o.z, acc.z);
+            acc.w = fmaf(w, o.w, acc.w);
+        }
+        *reinterpret_cast<float4*>(a.selfcond + static_cast<size_t>(n) * a.d + col) =
+            make_float4(acc.x * invL, acc.y * invL, acc.z * invL, acc.w * invL);
+    }
+}
+
+}  // namespace dg

@@ -1,0 +1,55 @@
+// Kernel argument blocks and kernel declarations shared by the launch code.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace dg {
+
+struct FusedArgs {
+    CUtensorMap map_h;   // h [N, d] bf16, box {64 cols, 128 rows}
+    CUtensorMap map_w;   // W [V, d] bf16, box {64 cols, 256 rows}
+    CUtensorMap map_e;   // E [V, d] bf16, box {64 cols, 64 rows}
+    CUtensorMap map_p;   // P scratch [n_groups*2*G*128, 256] bf16, box {64 cols, 128 rows}
+    const int32_t* stop;
+    uint32_t* counters;
+    float* rowmax;
+    __nv_bfloat16* pbuf;
+    float4* stats;
+    int32_t* stat_idx;
+    float* opart;
+    int* err;
+    int C, V, d, G, slice, n_groups, steps_per_tile, max_seg;
+    float scale_log2;    // log2(e) / T
+};
+
+struct CombineArgs {
+    const int32_t* stop;
+    uint32_t* counters;
+    const float4* stats;
+    const int32_t* stat_idx;
+    const float* opart;
+    float* entropy;
+    int32_t* argmax;
+    float* lse;
+    float* selfcond;
+    int C, d, G, n_groups, steps_per_tile, max_seg;
+};
+
+__global__ void dg_fused_kernel(const __grid_constant__ FusedArgs a);
+__global__ void dg_combine_kernel(const CombineArgs a);
+
+// small kernels (dg_small.cu)
+__global__ void dg_init_kernel(const uint64_t* seeds, int32_t* tokens, int32_t* prev_argmax, int32_t* stable,
+                               int32_t* stop, int32_t* err, uint32_t* counters, int n_counter_words, int C, int V);
+__global__ void dg_accept_kernel(const float* entropy, const int32_t* argmax, const uint64_t* seeds,
+                                 const int32_t* stop, int32_t* tokens, uint8_t* accept, float bound, int step,
+                                 int N, int V);
+__global__ void dg_stop_kernel(const float* entropy, const int32_t* argmax, int32_t* prev_argmax, int32_t* stable,
+                               int32_t* stop, float stop_thresh, int stability, int step);
+__global__ void dg_stub_kernel(const uint64_t* seeds, const __nv_bfloat16* E, const int32_t* tokens,
+                               const int32_t* stop, __nv_bfloat16* h, float a_s, float gain, float noise, int step,
+                               int d, int V, int N);
+
+}  // namespace dg

@@ -1,0 +1,165 @@
+/*
+ * dg.h - C ABI of the canvas denoise-sampling stage (uniform-state block
+ * diffusion, DiffusionGemma style) on NVIDIA B200 (sm_100a).
+ *
+ * What one step computes, for every position i of every active 256-token
+ * canvas c (pages: marrrang.tistory.com "DiffusionGemma deep dive", sections
+ * "Uniform State Diffusion", "reverse diffusion" steps 1-7, "standard sampling
+ * settings" table and "Two-Fold Adaptive Stopping"; juhoplayground.github.io
+ * "DiffusionGemma", section "inference mechanism"; axbrief.com "DiffusionGemma",
+ * --diffusion-eb-max-steps):
+ *
+ *   z[i,v]  = (h_i . W_v) / T_s                      vocabulary-head logits
+ *   p       = softmax(z_i), LSE_i = log sum_v e^{z}, H_i = LSE_i - sum_v p z   (nats)
+ *   a_i     = argmax_v z[i,v]  (smallest index on exact ties)
+ *   sc_i    = sum_v p[i,v] E_v                        self-conditioning vector
+ *   accept  = H_i <= bound; x_i <- accept ? a_i : Uniform(V) (Philox, tag 1)
+ *   stop_c  = mean_i H_i < stop_thresh  AND  argmax unchanged for `stability`
+ *             consecutive steps (stable counter, 0 at step 1)
+ *   T_s     = t_start + (t_end - t_start) (s-1)/(S-1), s = 1..S
+ *
+ * No N x V logits tensor is ever stored: one fused pass streams W and E.
+ *
+ * Conventions for every entry point:
+ *  - All pointers named *_dev are device pointers owned by the caller; the
+ *    library allocates and frees nothing and keeps no global state besides a
+ *    lazily resolved driver entry point and per-device attribute cache.
+ *  - Matrices are row-major and dense: h [N, d], W and E [V, d] (bf16),
+ *    selfcond [N, d] (fp32); N = n_canvas * canvas_len, positions of canvas c
+ *    are rows c*canvas_len .. c*canvas_len + canvas_len - 1.
+ *  - All calls are asynchronous on `stream` except dg_stop_check, which
+ *    synchronises that stream.  Argument errors are reported before anything
+ *    is launched.  Nothing throws across this boundary.
+ *  - A wait inside a kernel that runs past its time limit records an error
+ *    word in the workspace; the next dg_stop_check returns DG_ETIMEOUT.
+ *  - Philox4x32-10 (Salmon et al., SC'11) keys: key = (lo32(seed_c), hi32(seed_c)),
+ *    counter = (position within canvas, step, canvas index, tag); tag 0 canvas
+ *    init (step 0), 1 re-noise, 2 stub target ids, 3 stub Gaussian noise.
+ *    A token is floor(word0 * V / 2^32).
+ */
+#ifndef DG_H_
+#define DG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DG_OK = 0,
+    DG_EINVAL = -1,         /* bad argument (null pointer, bad size, bad step) */
+    DG_ECUDA = -2,          /* a CUDA runtime / driver call failed */
+    DG_EUNSUPPORTED = -3,   /* shape the kernels do not handle (see dg_params) */
+    DG_ETIMEOUT = -4,       /* a bounded in-kernel wait ran out (reported by dg_stop_check) */
+    DG_ENOMEM = -5          /* workspace smaller than dg_workspace_size() */
+} dg_status;
+
+/*
+ * Sampler configuration.  Defaults from the deep dive's settings table:
+ * max_steps 48, temperature 0.8 -> 0.4, entropy bound 0.1, stop threshold
+ * 0.005, stability 2.  Supported shapes: canvas_len == 256; vocab a multiple of
+ * 256 and < 2^31; hidden a multiple of 64 whose column slice width (hidden /
+ * group) is a multiple of 64 and at most 256, with group <= the SM count;
+ * 1 <= n_canvas <= 1024.
+ */
+typedef struct {
+    int n_canvas;       /* C: independent canvases processed together */
+    int canvas_len;     /* positions per canvas; must be 256 */
+    int vocab;          /* V */
+    int hidden;         /* d */
+    int max_steps;      /* S >= 1 */
+    float t_start;      /* temperature at step 1 */
+    float t_end;        /* temperature at step S */
+    float eb_bound;     /* accept when H <= eb_bound (nats) */
+    float stop_thresh;  /* stop needs mean H < stop_thresh (nats) */
+    int stability;      /* stop needs stable >= stability */
+    int tied;           /* informational: 1 when E_dev == W_dev */
+    int group;          /* column-slice group size of the fused kernel; 0 = automatic */
+} dg_params;
+
+/* Fill a dg_params with the pages' defaults for C canvases of a (V, d) head. */
+void dg_params_default(dg_params* p, int n_canvas, int vocab, int hidden);
+
+/* Temperature T_s used at step s (1-based), as the float the kernels receive. */
+float dg_temperature(const dg_params* p, int step);
+
+/*
+ * Bytes of device workspace dg_canvas_init / dg_denoise_step / dg_stop_check
+ * need for these params on the current device (the fused kernel's grid depends
+ * on the device's SM count).  Returns 0 if the params are invalid.
+ */
+size_t dg_workspace_size(const dg_params* p);
+
+/*
+ * Canvas initialisation (uniform-state noise, deep dive "reverse diffusion"
+ * step 1; juhoplayground "Entropy Bounded Sampler": start from uniform random
+ * tokens).  tokens_dev[c*256 + i] = Philox(seed_c; i, 0, c, 0) mapped to [0, V).
+ * Also resets the per-canvas state in the workspace (stable counters, stop
+ * flags, previous argmax, error word).
+ *   seeds_dev:  [C] uint64 device array.
+ *   tokens_dev: [C*256] int32 device array (written).
+ */
+dg_status dg_canvas_init(const dg_params* p, const uint64_t* seeds_dev, int32_t* tokens_dev,
+                         void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/*
+ * One denoising step s (1 <= s <= max_steps) of every canvas not yet stopped.
+ *   h_dev:        [N, d] bf16 hidden states of the denoiser (read).
+ *   W_dev, E_dev: [V, d] bf16 vocabulary head and token embedding (read);
+ *                 pass the same pointer for tied weights.
+ *   seeds_dev:    [C] uint64 (read).
+ *   tokens_dev:   [N] int32 canvas (read for inactive canvases, written for active).
+ *   entropy_dev:  [N] float, H in nats (written for active canvases).
+ *   argmax_dev:   [N] int32 (written for active canvases; for a stopped canvas
+ *                 it keeps the argmax of its last step, i.e. the committed block).
+ *   accept_dev:   [N] uint8 (written for active canvases).
+ *   lse_dev:      [N] float log-sum-exp of z (may be NULL).
+ *   selfcond_dev: [N, d] float (may be NULL: the fused kernel still computes it,
+ *                 only the final normalised copy is skipped).
+ * Canvases whose stop flag is set are skipped.  Step order inside: fused
+ * logits/softmax/entropy/argmax/self-conditioning pass, split-vocabulary
+ * combine, accept/re-noise, stop reduction.  The stop decision of step s is
+ * visible to dg_stop_check after this call.
+ */
+dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const void* W_dev,
+                          const void* E_dev, const uint64_t* seeds_dev, int32_t* tokens_dev,
+                          float* entropy_dev, int32_t* argmax_dev, uint8_t* accept_dev, float* lse_dev,
+                          float* selfcond_dev, void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/*
+ * The only host synchronisation point: waits for `stream`, copies the C stop
+ * flags into stop_flags_host (int32 [C], may be NULL) and the number of stopped
+ * canvases into *n_stopped_host (may be NULL), and reports a device-side
+ * timeout as DG_ETIMEOUT.  Optionally copies the per-canvas stable counters
+ * into stable_host (int32 [C], may be NULL).
+ */
+dg_status dg_stop_check(const dg_params* p, void* workspace_dev, size_t workspace_bytes, int32_t* stop_flags_host,
+                        int32_t* stable_host, int* n_stopped_host, void* stream);
+
+/*
+ * Benchmark-only stand-in for the denoiser network (not on the pages):
+ *   h_i = gain * (a E[tgt_i] + (1 - a) E[x_i]) + noise * n_i,   a = s / max_steps,
+ * tgt_i uniform over V (Philox tag 2, step 0), n_i standard normal by Box-Muller on
+ * Philox tag 3 words (counter (i*d/4 + k/4, s, c, 3)).  Computed in fp32, stored bf16.
+ * Only canvases not yet stopped are written (the workspace holds the flags).
+ */
+dg_status dg_stub_hidden(const dg_params* p, int step, float gain, float noise, const uint64_t* seeds_dev,
+                         const void* E_dev, const int32_t* tokens_dev, void* h_dev, void* workspace_dev,
+                         size_t workspace_bytes, void* stream);
+
+/* Static description of a status code. */
+const char* dg_status_string(dg_status s);
+
+/* Number of kernel launches the last dg_denoise_step on this thread issued. */
+int dg_last_launch_count(void);
+
+/* Column-slice group size and group count the fused kernel uses for p on the current device. */
+dg_status dg_plan(const dg_params* p, int* group, int* n_groups, int* slice_cols);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_H_ */

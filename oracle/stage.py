@@ -172,6 +172,44 @@ def denoise_step(h_u16, W_u16, E_u16, T, bound, seeds, s, vocab, canvas_len=256,
     return res
 
 
+# ------------------------------------------------------------ large vocabularies
+def logits_chunked(h, W_u16, T, chunk=16384):
+    """z = (h W^T) / T in float64, widening W chunk by chunk (memory only: same arithmetic as ``logits``)."""
+    h = np.asarray(h, np.float64)
+    V = W_u16.shape[0]
+    z = np.empty((h.shape[0], V))
+    for v0 in range(0, V, chunk):
+        v1 = min(V, v0 + chunk)
+        z[:, v0:v1] = (h @ bf16_to_f64(W_u16[v0:v1]).T) / float(T)
+    return z
+
+
+def self_conditioning_chunked(p, E_u16, chunk=16384):
+    """sc = p E in float64, widening E chunk by chunk (memory only)."""
+    V, d = E_u16.shape
+    sc = np.zeros((p.shape[0], d))
+    for v0 in range(0, V, chunk):
+        v1 = min(V, v0 + chunk)
+        sc += p[:, v0:v1] @ bf16_to_f64(E_u16[v0:v1])
+    return sc
+
+
+def step_rows(h_u16, W_u16, E_u16, T, bound, seed, s, c, positions, vocab, want_selfcond=True):
+    """One step for selected positions of one canvas (rows of h_u16 are those positions).
+
+    positions: index of each row within its canvas (for the re-noise draw).
+    Returns dict with H, argmax, lse, top2gap, tokens, accept, selfcond.
+    """
+    h = bf16_to_f64(h_u16)
+    st = distribution_stats(logits_chunked(h, W_u16, T))
+    ren = philox.uniform_token(seed, np.asarray(positions), s, c, philox.TAG_RENOISE, vocab)
+    tok, acc = eb_accept(st["H"], st["argmax"], bound, ren)
+    out = {k: st[k] for k in ("H", "argmax", "lse", "top2gap", "max")}
+    out["tokens"], out["accept"] = tok, acc
+    out["selfcond"] = self_conditioning_chunked(st["p"], E_u16) if want_selfcond else None
+    return out
+
+
 # ------------------------------------------------------- split-vocabulary statistics
 def partial_stats(z):
     """Statistics of one vocabulary range, relative to that range's own maximum.

@@ -1,0 +1,88 @@
+"""Helpers for the GPU parity tests: run the CUDA path through the C ABI binding,
+run the oracle on the same inputs, and compare under the stated tolerances.
+
+Tolerances (per position): H within 1e-3 nats; self-conditioning within 2e-2
+relative L2; tokens, accept flags and argmax bit-exact except at positions whose
+oracle entropy is within 1e-3 of the bound or whose top-2 logits (z = h.W/T)
+differ by less than 1e-3 - those are listed and excluded.
+"""
+
+import numpy as np
+import torch
+
+import synth
+from oracle import stage
+
+H_TOL = 1e-3
+SC_TOL = 2e-2
+EXCL = 1e-3
+
+
+def to_dev(t):
+    return t.to("cuda")
+
+
+def gpu_step(dg, p, step, h, Wd, Ed, seeds, tokens_in=None, ws=None, bufs=None):
+    """One dg_denoise_step on device tensors; returns host numpy outputs."""
+    ws = ws or dg.Workspace(p)
+    bufs = bufs or dg.StepBuffers(p)
+    seeds_t = torch.tensor(np.asarray(seeds, np.uint64).astype(np.int64), device="cuda")
+    dg.dg_canvas_init(p, seeds_t, bufs.tokens, ws)
+    if tokens_in is not None:
+        bufs.tokens.copy_(torch.as_tensor(np.asarray(tokens_in, np.int32)).cuda())
+    bufs.h.copy_(h.cuda() if not h.is_cuda else h)
+    dg.dg_denoise_step(p, step, bufs.h, Wd, Ed, seeds_t, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept,
+                       bufs.lse, bufs.selfcond, ws)
+    flags, stable, _ = dg.dg_stop_check(p, ws, want_stable=True)
+    out = {"H": bufs.entropy.cpu().numpy().astype(np.float64), "argmax": bufs.argmax.cpu().numpy().astype(np.int64),
+           "tokens": bufs.tokens.cpu().numpy().astype(np.int64), "accept": bufs.accept.cpu().numpy(),
+           "lse": bufs.lse.cpu().numpy().astype(np.float64),
+           "selfcond": bufs.selfcond.cpu().numpy().astype(np.float64) if bufs.selfcond is not None else None,
+           "stop": np.array(flags), "stable": np.array(stable)}
+    return out
+
+
+def oracle_rows(h_bits, W_bits, E_bits, T, bound, seeds, step, rows, vocab, canvas_len=256, want_selfcond=True):
+    """Oracle for selected global rows (positions); canvas index and seed derive from the row."""
+    rows = np.asarray(rows)
+    n, d = len(rows), h_bits.shape[1]
+    out = {"H": np.empty(n), "argmax": np.empty(n, np.int64), "lse": np.empty(n), "top2gap": np.empty(n),
+           "tokens": np.empty(n, np.int64), "accept": np.empty(n, np.uint8),
+           "selfcond": np.empty((n, d)) if want_selfcond else None}
+    for c in np.unique(rows // canvas_len):
+        idx = np.nonzero(rows // canvas_len == c)[0]
+        r = stage.step_rows(h_bits[rows[idx]], W_bits, E_bits, T, bound, int(seeds[c]), step, int(c),
+                            rows[idx] % canvas_len, vocab, want_selfcond)
+        for k in out:
+            if out[k] is not None:
+                out[k][idx] = r[k]
+    return out
+
+
+def compare(gpu, ora, rows, bound, check_selfcond=True, tag=""):
+    """Assert parity on `rows`; returns (excluded row list, max H error, max sc error)."""
+    H = gpu["H"][rows]
+    dH = np.abs(H - ora["H"])
+    excl = (np.abs(ora["H"] - bound) < EXCL) | (ora["top2gap"] < EXCL)
+    assert np.all(np.isfinite(H)), f"{tag}: non-finite entropy"
+    assert dH.max() <= H_TOL, f"{tag}: max |dH| = {dH.max():.3e} at row {rows[int(dH.argmax())]}"
+    ok = ~excl
+    bad = np.nonzero(ok & (gpu["argmax"][rows] != ora["argmax"]))[0]
+    assert bad.size == 0, f"{tag}: argmax mismatch at rows {rows[bad][:8]}"
+    bad = np.nonzero(ok & (gpu["accept"][rows] != ora["accept"]))[0]
+    assert bad.size == 0, f"{tag}: accept mismatch at rows {rows[bad][:8]}"
+    bad = np.nonzero(ok & (gpu["tokens"][rows] != ora["tokens"]))[0]
+    assert bad.size == 0, f"{tag}: token mismatch at rows {rows[bad][:8]}"
+    dl = np.abs(gpu["lse"][rows] - ora["lse"])
+    assert dl.max() <= 1e-3 * np.maximum(1.0, np.abs(ora["lse"])).max(), f"{tag}: lse error {dl.max():.3e}"
+    esc = 0.0
+    if check_selfcond and gpu["selfcond"] is not None and ora["selfcond"] is not None:
+        a, b = gpu["selfcond"][rows], ora["selfcond"]
+        rel = np.linalg.norm(a - b, axis=1) / np.maximum(np.linalg.norm(b, axis=1), 1e-30)
+        esc = float(rel.max())
+        assert esc <= SC_TOL, f"{tag}: self-conditioning rel L2 {esc:.3e} at row {rows[int(rel.argmax())]}"
+    return rows[excl].tolist(), float(dH.max()), esc
+
+
+def bits(t):
+    return synth.bf16_bits(t.cpu())

@@ -1,0 +1,65 @@
+"""The C ABI library builds, loads and exports every symbol include/dg.h declares (CPU only).
+
+No compute call is made here: only host-side helpers that touch no device.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dg.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dg_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from discrete_diffusion_decoding_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    for n in ("dg_canvas_init", "dg_denoise_step", "dg_stop_check", "dg_stub_hidden", "dg_workspace_size"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, f"not exported: {missing}"
+
+
+def test_binding_covers_the_header():
+    from discrete_diffusion_decoding_b200 import _abi
+    assert sorted(_abi.EXPORTS) == _declared()
+
+
+def test_host_helpers_without_device(lib):
+    from discrete_diffusion_decoding_b200 import _abi
+    p = _abi.DgParams()
+    lib.dg_params_default.argtypes = [ctypes.POINTER(_abi.DgParams), ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.dg_params_default(ctypes.byref(p), 16, 262144, 2816)
+    assert (p.n_canvas, p.canvas_len, p.vocab, p.hidden, p.max_steps) == (16, 256, 262144, 2816, 48)
+    assert abs(p.t_start - 0.8) < 1e-7 and abs(p.t_end - 0.4) < 1e-7
+    assert abs(p.eb_bound - 0.1) < 1e-7 and abs(p.stop_thresh - 0.005) < 1e-9 and p.stability == 2
+    lib.dg_temperature.argtypes = [ctypes.POINTER(_abi.DgParams), ctypes.c_int]
+    lib.dg_temperature.restype = ctypes.c_float
+    from oracle import stage
+    for s in (1, 2, 17, 48):
+        assert lib.dg_temperature(ctypes.byref(p), s) == stage.temperature(s, 48)
+    lib.dg_status_string.restype = ctypes.c_char_p
+    assert lib.dg_status_string(-4) == b"in-kernel wait timed out"
+
+
+def test_sm100a_only_build():
+    from discrete_diffusion_decoding_b200 import build
+    src = open(build.__file__).read()
+    assert "arch=compute_100a,code=sm_100a" in src

@@ -1,0 +1,306 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Every test here runs the library's sm_100a kernels on a B200 and compares with
+the oracle on the same seeded inputs (see gpu_case.py for the tolerances).
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import gpu_case as gc
+import synth
+from oracle import philox, stage
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dg():
+    from discrete_diffusion_decoding_b200 import build
+    build.build()
+    import discrete_diffusion_decoding_b200 as m
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return m
+
+
+@pytest.fixture(scope="module")
+def big_W():
+    W = synth.weights(262144, 2816, seed=1234)
+    return W, gc.bits(W), W.cuda()
+
+
+def _assert_stub_close(got_bits, want_bits, gain):
+    # one bf16 ulp of the result, plus the fp32 rounding of the sum's operands (which may cancel)
+    a_got = stage.bf16_to_f64(got_bits)
+    a_want = stage.bf16_to_f64(want_bits)
+    ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(a_want), 2.0 ** -120))) - 7)
+    err = np.abs(a_got - a_want)
+    assert np.all(err <= ulp + 1e-6 * max(1.0, gain)), f"stub error {err.max():.3e}"
+    assert (err == 0).mean() > 0.99
+
+
+def _rows_all(n):
+    return np.arange(n)
+
+
+# ------------------------------------------------------------------ element-wise kernels
+def test_canvas_init_bitexact(dg):
+    V = 262144
+    C = 1024                                   # 262144 Philox draws
+    p = dg.params(C, V, 128)
+    seeds = (np.arange(C, dtype=np.uint64) * np.uint64(0x9E3779B97F4A7C15)) + np.uint64(7)
+    ws = dg.Workspace(p)
+    tok = torch.empty(C * 256, dtype=torch.int32, device="cuda")
+    dg.dg_canvas_init(p, torch.tensor(seeds.view(np.int64), device="cuda"), tok, ws)
+    got = tok.cpu().numpy()
+    want = np.concatenate([stage.init_tokens(int(seeds[c]), c, V) for c in range(C)])
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("V,d,C,gain,noise,step,S", [(4096, 128, 2, 300.0, 0.1, 5, 16),
+                                                      (262144, 2816, 1, 8.0, 0.1, 48, 48)])
+def test_stub_hidden_within_one_ulp(dg, V, d, C, gain, noise, step, S):
+    W = synth.weights(V, d)
+    Wb = gc.bits(W)
+    p = dg.params(C, V, d, max_steps=S)
+    seeds = synth.canvas_seeds(C, base=11)
+    rng = np.random.default_rng(3)
+    toks = rng.integers(0, V, size=C * 256).astype(np.int32)
+    ws = dg.Workspace(p)
+    Wd = W.cuda()
+    seeds_t = torch.tensor(seeds.view(np.int64), device="cuda")
+    tok_t = torch.tensor(toks, device="cuda")
+    dg.dg_canvas_init(p, seeds_t, torch.empty_like(tok_t), ws)
+    h = torch.empty((C * 256, d), dtype=torch.bfloat16, device="cuda")
+    dg.dg_stub_hidden(p, step, gain, noise, seeds_t, Wd, tok_t, h, ws)
+    got = gc.bits(h)
+    for c in range(C):
+        want, _ = stage.stub_hidden(Wb, toks[c * 256:(c + 1) * 256], int(seeds[c]), step, c, S, gain, noise)
+        _assert_stub_close(got[c * 256:(c + 1) * 256], want, gain)
+
+
+# ------------------------------------------------------------------ one step, small shapes
+@pytest.mark.parametrize("kind", ["gaussian", "spiked"])
+def test_step_small_tied(dg, kind):
+    V, d, C = 4096, 128, 1
+    W = synth.weights(V, d)
+    h = synth.gaussian_hidden(C * 256, d, seed=42) if kind == "gaussian" else synth.spiked_hidden(W, C * 256, gain_lo=0.5, gain_hi=20.0)[0]
+    p = dg.params(C, V, d)
+    seeds = synth.canvas_seeds(C)
+    Wd = W.cuda()
+    g = gc.gpu_step(dg, p, 1, h, Wd, Wd, seeds)
+    T = dg.temperature(p, 1)
+    o = gc.oracle_rows(gc.bits(h), gc.bits(W), gc.bits(W), T, p.eb_bound, seeds, 1, _rows_all(C * 256), V)
+    excl, dh, dsc = gc.compare(g, o, _rows_all(C * 256), p.eb_bound, tag=kind)
+    assert len(excl) < 32
+    if kind == "spiked":
+        assert 0 < int(g["accept"].sum()) < C * 256           # both branches of the sampler taken
+
+
+@pytest.mark.parametrize("group,tied,C,V", [(2, True, 2, 8960), (4, False, 2, 8960), (8, True, 3, 4096),
+                                            (1, True, 2, 65536)])
+def test_step_groups_and_segments(dg, group, tied, C, V):
+    """Multi-CTA groups (P exchange, shared reference), tile-spanning segments, ragged blocks."""
+    d = 512 if group > 1 else 256
+    W = synth.weights(V, d, seed=1234)
+    E = W if tied else synth.weights(V, d, seed=1235)
+    h, _ = synth.spiked_hidden(W, C * 256, seed=50 + group, gain_lo=0.5, gain_hi=30.0)
+    p = dg.params(C, V, d, group=group, tied=int(tied))
+    seeds = synth.canvas_seeds(C, base=100)
+    Wd = W.cuda()
+    Ed = Wd if tied else E.cuda()
+    g = gc.gpu_step(dg, p, 3, h, Wd, Ed, seeds)
+    T = dg.temperature(p, 3)
+    o = gc.oracle_rows(gc.bits(h), gc.bits(W), gc.bits(E), T, p.eb_bound, seeds, 3, _rows_all(C * 256), V)
+    gc.compare(g, o, _rows_all(C * 256), p.eb_bound, tag=f"G={group}")
+
+
+def test_large_logits_rescale(dg):
+    """Rows whose running maximum jumps late in the vocabulary force the lazy rescale of O."""
+    V, d, C = 131072, 512, 1          # G = 2: 256 blocks per tile, several blocks per segment
+    W = synth.weights(V, d, seed=9)
+    Wf = W.to(torch.float64)
+    h = torch.zeros((256, d), dtype=torch.float64)
+    g = torch.Generator().manual_seed(5)
+    for i in range(256):
+        k = int(torch.randint(0, V, (1,), generator=g))       # the spike's block is usually not a segment's first
+        h[i] = Wf[k] * ((10.0 + 0.3 * (i % 90)) / float(Wf[k] @ Wf[k]))
+    h = h.to(torch.float32).to(torch.bfloat16)
+    p = dg.params(C, V, d, group=2)
+    seeds = synth.canvas_seeds(C)
+    Wd = W.cuda()
+    out = gc.gpu_step(dg, p, 1, h, Wd, Wd, seeds)
+    o = gc.oracle_rows(gc.bits(h), gc.bits(W), gc.bits(W), dg.temperature(p, 1), p.eb_bound, seeds, 1,
+                       _rows_all(256), V)
+    gc.compare(out, o, _rows_all(256), p.eb_bound, tag="rescale")
+
+
+def test_uniform_logits_closed_form(dg):
+    """h = 0: every logit ties, H = ln V, argmax = 0, self-conditioning = column mean of E."""
+    V, d, C = 8192, 512, 1
+    W = synth.weights(V, d)
+    p = dg.params(C, V, d)
+    h = torch.zeros((256, d), dtype=torch.bfloat16)
+    Wd = W.cuda()
+    g = gc.gpu_step(dg, p, 1, h, Wd, Wd, synth.canvas_seeds(1))
+    assert np.abs(g["H"] - math.log(V)).max() < 1e-4
+    assert np.all(g["argmax"] == 0)
+    mean = stage.bf16_to_f64(gc.bits(W)).mean(axis=0)
+    rel = np.linalg.norm(g["selfcond"] - mean[None, :], axis=1) / np.linalg.norm(mean)
+    assert rel.max() < 1e-3
+
+
+# ------------------------------------------------------------------ full-size single step
+def _sample_rows(N, n, seed):
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, 127, 128, 255, N - 1]
+    return np.unique(np.concatenate([fixed, rng.choice(N, size=n, replace=False)]))
+
+
+@pytest.mark.parametrize("hidden_kind,step,S", [("gaussian", 1, 48), ("spiked", 48, 48)])
+def test_full_vocab_single_step(dg, big_W, hidden_kind, step, S):
+    W, Wb, Wd = big_W
+    V, d, C = 262144, 2816, 1
+    if hidden_kind == "gaussian":
+        h = synth.gaussian_hidden(256, d, seed=42)
+    else:
+        h, _ = synth.spiked_hidden(W, 256, seed=43, gain_lo=2.0, gain_hi=40.0)
+    p = dg.params(C, V, d, max_steps=S)
+    seeds = synth.canvas_seeds(C)
+    g = gc.gpu_step(dg, p, step, h, Wd, Wd, seeds)
+    rows = _sample_rows(256, 40, 1)
+    o = gc.oracle_rows(gc.bits(h), Wb, Wb, dg.temperature(p, step), p.eb_bound, seeds, step, rows, V)
+    gc.compare(g, o, rows, p.eb_bound, tag=hidden_kind)
+    # properties that hold at every position
+    assert np.all(g["H"] >= -1e-4) and np.all(g["H"] <= math.log(V) + 1e-3)
+    assert np.all((g["argmax"] >= 0) & (g["argmax"] < V))
+
+
+def test_batched_full_vocab_step(dg, big_W):
+    """16 canvases (N = 4096) in one launch, per-canvas seeds: sampled rows in every canvas."""
+    W, Wb, Wd = big_W
+    V, d, C = 262144, 2816, 16
+    h, _ = synth.spiked_hidden(W, C * 256, seed=60, gain_lo=2.0, gain_hi=40.0)
+    p = dg.params(C, V, d)
+    seeds = synth.canvas_seeds(C, base=1000)
+    g = gc.gpu_step(dg, p, 7, h, Wd, Wd, seeds)
+    rows = _sample_rows(C * 256, 48, 2)
+    o = gc.oracle_rows(gc.bits(h), Wb, Wb, dg.temperature(p, 7), p.eb_bound, seeds, 7, rows, V)
+    gc.compare(g, o, rows, p.eb_bound, tag="batched")
+
+
+# ------------------------------------------------------------------ multi-step, lock-step
+def _lockstep(dg, V, d, C, S, gain, noise, seeds, W, sample=None, expect_stop=True):
+    p = dg.params(C, V, d, max_steps=S)
+    Wb = gc.bits(W)
+    Wd = W.cuda()
+    ws = dg.Workspace(p)
+    bufs = dg.StepBuffers(p)
+    seeds_t = torch.tensor(np.asarray(seeds, np.uint64).view(np.int64), device="cuda")
+    dg.dg_canvas_init(p, seeds_t, bufs.tokens, ws)
+    init = bufs.tokens.cpu().numpy()
+    for c in range(C):
+        assert np.array_equal(init[c * 256:(c + 1) * 256], stage.init_tokens(int(seeds[c]), c, V))
+    prev = [None] * C
+    stable = [0] * C
+    stopped = [False] * C
+    stop_at = [S] * C
+    for s in range(1, S + 1):
+        tok_in = bufs.tokens.cpu().numpy().copy()
+        dg.dg_stub_hidden(p, s, gain, noise, seeds_t, Wd, bufs.tokens, bufs.h, ws)
+        dg.dg_denoise_step(p, s, bufs.h, Wd, Wd, seeds_t, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept,
+                           bufs.lse, bufs.selfcond, ws)
+        flags, st_gpu, _ = dg.dg_stop_check(p, ws, want_stable=True)
+        hb = gc.bits(bufs.h)
+        g = {"H": bufs.entropy.cpu().numpy().astype(np.float64), "argmax": bufs.argmax.cpu().numpy().astype(np.int64),
+             "tokens": bufs.tokens.cpu().numpy().astype(np.int64), "accept": bufs.accept.cpu().numpy(),
+             "lse": bufs.lse.cpu().numpy().astype(np.float64), "selfcond": bufs.selfcond.cpu().numpy()}
+        T = dg.temperature(p, s)
+        for c in range(C):
+            if stopped[c]:
+                continue
+            rows_c = np.arange(c * 256, (c + 1) * 256)
+            # the stub is an input of the stage: check it, then hand its bytes to the oracle
+            want_h, _ = stage.stub_hidden(Wb, tok_in[rows_c], int(seeds[c]), s, c, S, gain, noise)
+            _assert_stub_close(hb[rows_c], want_h, gain)
+            rows = rows_c if sample is None else rows_c[sample]
+            o = gc.oracle_rows(hb, Wb, Wb, T, p.eb_bound, seeds, s, rows, V)
+            excl, _, _ = gc.compare(g, o, rows, p.eb_bound, tag=f"s={s} c={c}")
+            if sample is None:
+                full = stage.distribution_stats(stage.logits_chunked(stage.bf16_to_f64(hb[rows_c]), Wb, T))
+                mean_H = full["H"].mean()
+                stable[c], stop = stage.stop_update(mean_H, g["argmax"][rows_c], prev[c], stable[c], s)
+                prev[c] = g["argmax"][rows_c].copy()
+                if not excl and abs(mean_H - p.stop_thresh) >= 1e-3:
+                    assert st_gpu[c] == stable[c], f"stable counter s={s} c={c}"
+                    assert bool(flags[c]) == stop, f"stop flag s={s} c={c}"
+            if flags[c]:
+                stopped[c] = True
+                stop_at[c] = s
+        if all(stopped):
+            break
+    if expect_stop:
+        assert min(stop_at) < S, "no canvas stopped early: the stop path was not exercised"
+    for c in range(C):
+        if stop_at[c] < S:
+            assert stop_at[c] >= 3
+    return stop_at
+
+
+def test_lockstep_decode_small(dg):
+    W = synth.weights(4096, 128)
+    stop_at = _lockstep(dg, 4096, 128, 1, 16, 300.0, 0.1, synth.canvas_seeds(1), W)
+    assert stop_at[0] <= 16
+
+
+def test_lockstep_batched_per_canvas_stop(dg):
+    W = synth.weights(4096, 128)
+    stop_at = _lockstep(dg, 4096, 128, 4, 16, 300.0, 0.1, synth.canvas_seeds(4, base=20), W)
+    assert len(set(stop_at)) >= 1
+
+
+def test_lockstep_literal_gain_never_accepts(dg):
+    """The literal small configuration (gain 1): entropies stay near ln V, nothing is accepted."""
+    W = synth.weights(4096, 128)
+    stop_at = _lockstep(dg, 4096, 128, 1, 4, 1.0, 0.1, synth.canvas_seeds(1), W, expect_stop=False)
+    assert stop_at == [4]
+
+
+# ------------------------------------------------------------------ argument checks
+def test_argument_errors(dg):
+    from discrete_diffusion_decoding_b200 import _abi
+    p = dg.params(1, 4096, 128)
+    ws = dg.Workspace(p)
+    bufs = dg.StepBuffers(p)
+    W = synth.weights(4096, 128).cuda()
+    seeds = torch.zeros(1, dtype=torch.int64, device="cuda")
+    with pytest.raises(_abi.DgError) as e:
+        dg.dg_denoise_step(p, 0, bufs.h, W, W, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept, None,
+                           None, ws)
+    assert e.value.status == _abi.DG_EINVAL
+    with pytest.raises(_abi.DgError) as e:
+        dg.dg_denoise_step(p, 49, bufs.h, W, W, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept, None,
+                           None, ws)
+    assert e.value.status == _abi.DG_EINVAL
+    with pytest.raises(_abi.DgError) as e:
+        dg.dg_denoise_step(p, 1, None, W, W, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept, None, None,
+                           ws)
+    assert e.value.status == _abi.DG_EINVAL
+    small = dg.Workspace(p)
+    small.nbytes = 64
+    with pytest.raises(_abi.DgError) as e:
+        dg.dg_denoise_step(p, 1, bufs.h, W, W, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept, None,
+                           None, small)
+    assert e.value.status == _abi.DG_ENOMEM
+    with pytest.raises(_abi.DgError):
+        dg.workspace_size(dg.params(1, 4000, 128))            # vocab not a multiple of 256
+    with pytest.raises(_abi.DgError):
+        dg.workspace_size(dg.params(1, 4096, 100))            # hidden not a multiple of 64
+    bad = dg.params(1, 4096, 512, group=3)
+    with pytest.raises(_abi.DgError) as e:
+        dg.plan(bad)
+    assert e.value.status == _abi.DG_EUNSUPPORTED
+    assert dg.last_launch_count() == 0
