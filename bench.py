@@ -1,0 +1,380 @@
+"""Benchmark of the canvas denoise-sampling stage on B200.
+
+Workload (the single-step microbenchmark): one 256-position canvas, vocabulary
+V = 262144, hidden d = 2816, tied bf16 head/embedding W = E ~ N(0, 0.02), hidden
+states N(0, 1) / sqrt(d) * 8, step 1 (T = 0.8), entropy bound 0.1.  A timed step
+is one dg_denoise_step: the fused logits / softmax / entropy / argmax /
+self-conditioning kernel, the split-vocabulary combine, accept / re-noise and the
+stop reduction.  Inputs are larger than L2 (W streams 1.48 GB per step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  With --gpus N > 1 (under torchrun) every rank
+runs an independent replica (canvases shard across GPUs with no data-path
+collective); the value is all ranks' positions over the slowest rank's time.
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+V, D, N_POS, STEP, BOUND = 262144, 2816, 256, 1, 0.1
+METRIC = "canvas positions/s per denoise step (V=262144,d=2816); % of roofline"
+WORKLOAD = ("single-step microbenchmark: 1 canvas of 256 positions, V=262144, d=2816, tied bf16 E=W ~N(0,0.02), "
+            "hidden bf16 N(0,1)/sqrt(d)*8, step 1 (T=0.8), bound 0.1; outputs tokens/H/argmax/accept/self-cond fp32")
+FLOPS_PER_STEP = 2 * (2.0 * N_POS * V * D)          # two contractions: logits and self-conditioning
+WE_BYTES_PER_STEP = 2.0 * V * D                     # tied bf16 W = E streamed once
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "dg_fused_kernel_single_step_v262144_d2816.md")
+FUSED_SRC = os.path.join(ROOT, "discrete_diffusion_decoding_b200", "csrc", "dg_fused.cu")
+
+
+def _set_vocab(vocab):
+    """Reduced-vocabulary variant of the workload (profiler captures only)."""
+    global V, FLOPS_PER_STEP, WE_BYTES_PER_STEP, WORKLOAD
+    V = int(vocab)
+    FLOPS_PER_STEP = 2 * (2.0 * N_POS * V * D)
+    WE_BYTES_PER_STEP = 2.0 * V * D
+    WORKLOAD = WORKLOAD.replace("V=262144", f"V={V} (reduced, profiling only)")
+
+
+# ----------------------------------------------------------------------------- helpers
+def dist_env():
+    """(rank, world_size, local_rank) from the torchrun environment (1-process defaults)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def shard_canvases(n_canvas_total, rank, world):
+    """Contiguous canvas range of one rank (replicas: every rank gets its own canvases)."""
+    lo = (n_canvas_total * rank) // world
+    hi = (n_canvas_total * (rank + 1)) // world
+    return lo, hi
+
+
+def max_over_ranks(value, backend_device=None):
+    """Maximum of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as tdist
+    if not (tdist.is_available() and tdist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=backend_device or "cpu")
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def profiled_traffic():
+    """DRAM bytes per fused launch from the committed ncu summary, if it was taken on this kernel source."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+        src_hash = hashlib.sha256(open(FUSED_SRC, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    fields = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("kernel_source_sha256") != src_hash:
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        self.dev = device_index
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            ident = self._nvsmi_id()
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", ident, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _nvsmi_id(self):
+        import torch
+        try:
+            pr = torch.cuda.get_device_properties(self.dev)
+            return f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            return vis.split(",")[self.dev] if vis else str(self.dev)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, st in rows for i, v in enumerate(st) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+def oracle_sample_rate(W64, h_bits, n_rows, T):
+    """Time the float64 oracle on n_rows positions of the workload; returns (positions/s, seconds, threads).
+
+    W64 is the head widened to float64 once, outside the timed call.
+    """
+    from oracle import stage
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    stage.step_rows(h_bits[:n_rows], W64, W64, T, BOUND, 0, STEP, 0, list(range(n_rows)), V)
+    dt = time.perf_counter() - t0
+    return n_rows / dt, dt, threads
+
+
+def run_reference(args):
+    """--impl reference: the float64 CPU oracle as it stands, timed on the host cores."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import synth
+    from oracle import stage
+    W = synth.weights(V, D, seed=1234)
+    h = synth.gaussian_hidden(N_POS, D, seed=42)
+    W64, hb = stage.bf16_to_f64(synth.bf16_bits(W)), synth.bf16_bits(h)
+    del W
+    T = stage.temperature(STEP, 48)
+    # bounded sample per step: size it from one probe so the whole run stays within about two minutes
+    _, probe_dt, _ = oracle_sample_rate(W64, hb, 1, T)
+    n_rows = int(max(1, min(N_POS, 120.0 / max(1, args.steps + args.warmup) / probe_dt)))
+    for _ in range(args.warmup):
+        oracle_sample_rate(W64, hb, 1, T)
+    times, threads = [], 1
+    for _ in range(args.steps):
+        rate, dt, threads = oracle_sample_rate(W64, hb, n_rows, T)
+        times.append(dt)
+    ms = statistics.mean(times) * 1e3 * (N_POS / n_rows)     # scaled to a full 256-position step
+    value = N_POS / (ms * 1e-3)
+    line = {"metric": METRIC, "value": value, "unit": "positions/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "n_canvas": 1, "positions": N_POS, "vocab": V, "hidden": D},
+            "cpu_baseline": {"value": value, "unit": "positions/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{n_rows} of 256 positions per step, scaled to a full step"},
+            "e2e": {"value": value, "unit": "positions/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU leg
+def run_gpu(args):
+    import numpy as np
+    import torch
+    import torch.distributed as tdist
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        tdist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+
+    import synth
+    from discrete_diffusion_decoding_b200 import build
+    build.build()
+    import discrete_diffusion_decoding_b200 as dg
+
+    # replicas: every rank owns one canvas of its own (seed = its global canvas index)
+    c0, _ = shard_canvases(world, rank, world)
+    p = dg.params(1, V, D)
+    W = synth.weights(V, D, seed=1234).to(dev)
+    h_host = synth.gaussian_hidden(N_POS, D, seed=42)
+    ws = dg.Workspace(p, dev)
+    bufs = dg.StepBuffers(p, dev)
+    seeds = torch.tensor([c0], dtype=torch.int64, device=dev)
+    dg.dg_canvas_init(p, seeds, bufs.tokens, ws)
+    bufs.h.copy_(h_host.to(dev))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        dg.dg_denoise_step(p, STEP, bufs.h, W, W, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept,
+                           bufs.lse, bufs.selfcond, ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    _, _, _ = dg.dg_stop_check(p, ws)
+    launches_per_step = dg.last_launch_count()
+
+    # ---- device-timed region: K steps, inputs resident, W (1.48 GB) larger than L2
+    if world > 1:
+        tdist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dg.profile_enable(args.steps)
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    n_k1, k1_ms, _ = dg.profile_collect()
+    if world > 1:
+        tdist.barrier()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    flags, _, _ = dg.dg_stop_check(p, ws)             # also surfaces an in-kernel timeout
+    elapsed_max = max_over_ranks(elapsed_ms, dev if world > 1 else None)
+    k1_max = max_over_ranks(k1_ms, dev if world > 1 else None)
+    ms_per_step = elapsed_max / args.steps
+
+    # ---- end to end through the public API: pinned host h in, results out, every step
+    h_pin = h_host.pin_memory()
+    out_H = torch.empty(N_POS, dtype=torch.float32).pin_memory()
+    out_tok = torch.empty(N_POS, dtype=torch.int32).pin_memory()
+    out_am = torch.empty(N_POS, dtype=torch.int32).pin_memory()
+    out_acc = torch.empty(N_POS, dtype=torch.uint8).pin_memory()
+    out_sc = torch.empty((N_POS, D), dtype=torch.float32).pin_memory()
+    e2e_steps = max(3, min(args.steps, 200))
+
+    def e2e_step():
+        bufs.h.copy_(h_pin, non_blocking=True)
+        step()
+        out_H.copy_(bufs.entropy, non_blocking=True)
+        out_tok.copy_(bufs.tokens, non_blocking=True)
+        out_am.copy_(bufs.argmax, non_blocking=True)
+        out_acc.copy_(bufs.accept, non_blocking=True)
+        out_sc.copy_(bufs.selfcond, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    if world > 1:
+        tdist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev if world > 1 else None) / e2e_steps
+    h2d = h_pin.numel() * h_pin.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in (out_H, out_tok, out_am, out_acc, out_sc))
+
+    line = None
+    if rank == 0:
+        peaks, peaks_src = load_peaks()
+        peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        peak_tf_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        achieved = FLOPS_PER_STEP / (k1_max * 1e-3) / 1e12
+        roof_ms = max(FLOPS_PER_STEP / (peak_tf * 1e12), WE_BYTES_PER_STEP / (float(peaks.get("hbm_gbs", 6650.0)) * 1e9)) * 1e3
+        traffic = profiled_traffic()
+        value = world * N_POS / (ms_per_step * 1e-3)
+        line = {
+            "metric": METRIC, "value": value, "unit": "positions/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "n_canvas": world, "positions": world * N_POS, "vocab": V, "hidden": D,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (W/E 1.48 GB streamed per step)",
+                       "group": dg.plan(p)["group"], "n_groups": dg.plan(p)["n_groups"]},
+            "steps_per_s": 1e3 / ms_per_step,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": achieved / peak_tf, "traffic": traffic,
+                         "kernel": "dg_fused_kernel", "kernel_ms": k1_max, "launches_timed": n_k1,
+                         "flops_per_launch": FLOPS_PER_STEP, "peak_source": f"{peaks_src} bf16 burst",
+                         "frac_of_sustained": achieved / peak_tf_sus,
+                         "step_frac": roof_ms / ms_per_step, "roofline_step_ms": roof_ms},
+            "e2e": {"value": world * N_POS / (e2e_ms * 1e-3), "unit": "positions/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+            "stop_flags_after": flags,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            # bounded sample of the same workload through the float64 oracle on the host cores
+            from oracle import stage
+            W64 = stage.bf16_to_f64(synth.bf16_bits(W.cpu()))
+            hb = synth.bf16_bits(h_host)
+            rate, dt, threads = oracle_sample_rate(W64, hb, args.cpu_rows, stage.temperature(STEP, 48))
+            del W64
+            line["cpu_baseline"] = {"value": rate, "unit": "positions/s", "cores": threads, "kind": "oracle",
+                                    "sample": f"{args.cpu_rows} of 256 positions of one step ({dt:.1f} s)"}
+    if world > 1:
+        tdist.barrier()
+        tdist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-rows", type=int, default=256, help="positions in the oracle's bounded CPU sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--vocab", type=int, default=262144,
+                    help="vocabulary size; smaller values are for profiler captures only, not bench lines")
+    args = ap.parse_args(argv)
+    if args.vocab != V:
+        _set_vocab(args.vocab)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -14,7 +14,8 @@ from . import _abi
 from ._abi import DgError, DgParams, check, lib
 
 __all__ = ["DgError", "DgParams", "params", "workspace_size", "plan", "temperature", "dg_canvas_init",
-           "dg_denoise_step", "dg_stop_check", "dg_stub_hidden", "last_launch_count", "Workspace",
+           "dg_denoise_step", "dg_stop_check", "dg_stub_hidden", "last_launch_count", "profile_enable",
+           "profile_collect", "Workspace", "StepBuffers",
            "decode_batch", "decode_block_ar"]
 
 
@@ -44,6 +45,18 @@ def plan(p):
 
 def temperature(p, step):
     return float(lib().dg_temperature(ctypes.byref(p), int(step)))
+
+
+def profile_enable(max_records):
+    """Record CUDA events around the next fused-kernel launches (measurement only)."""
+    check("dg_profile_enable", lib().dg_profile_enable(int(max_records)))
+
+
+def profile_collect():
+    """(launches recorded, mean ms, total ms) of the fused kernel since profile_enable."""
+    n, mean, tot = ctypes.c_int(), ctypes.c_float(), ctypes.c_float()
+    check("dg_profile_collect", lib().dg_profile_collect(ctypes.byref(n), ctypes.byref(mean), ctypes.byref(tot)))
+    return n.value, mean.value, tot.value
 
 
 def last_launch_count():

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/dg.h"
 #include "dg_common.cuh"
@@ -17,6 +18,24 @@ namespace {
 
 constexpr int kFusedSmem = 4 * 48 * 1024 + 1024 + 4 * kMaxCanvas;
 thread_local int g_last_launches = 0;
+
+// Event pairs recorded around fused-kernel launches while profiling is enabled.
+struct ProfileState {
+    bool on = false;
+    int max_records = 0;
+    std::vector<cudaEvent_t> start, stop;
+    int used = 0;
+};
+thread_local ProfileState g_prof;
+
+void profile_release() {
+    for (auto e : g_prof.start) cudaEventDestroy(e);
+    for (auto e : g_prof.stop) cudaEventDestroy(e);
+    g_prof.start.clear();
+    g_prof.stop.clear();
+    g_prof.used = 0;
+    g_prof.on = false;
+}
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -81,9 +100,12 @@ dg_status make_plan(const dg_params* p, int sms, Plan* pl) {
     q.slice = slice;
     q.n_groups = sms / G;
     q.steps_per_tile = (p->vocab + G * kBV - 1) / (G * kBV);
-    const long long U = 2LL * q.C * q.steps_per_tile;
-    const long long per_group = (U + q.n_groups - 1) / q.n_groups;
-    q.max_seg = static_cast<int>((per_group + q.steps_per_tile - 1) / q.steps_per_tile) + 1;
+    // partial slots per group: the most pieces any active-tile count can give a group
+    q.max_seg = 1;
+    for (int n_pt = 2; n_pt <= 2 * q.C; n_pt += 2) {
+        const int pg = pieces_per_group(n_pt, q.n_groups);
+        if (pg > q.max_seg) q.max_seg = pg;
+    }
     q.n_slots = q.n_groups * q.max_seg;
     *pl = q;
     return DG_OK;
@@ -261,7 +283,13 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    const bool prof = g_prof.on && g_prof.used < g_prof.max_records;
+    if (prof && cudaEventRecord(g_prof.start[g_prof.used], s) != cudaSuccess) return DG_ECUDA;
     if (cudaLaunchKernelEx(&cfg, dg_fused_kernel, fa) != cudaSuccess) return DG_ECUDA;
+    if (prof) {
+        if (cudaEventRecord(g_prof.stop[g_prof.used], s) != cudaSuccess) return DG_ECUDA;
+        ++g_prof.used;
+    }
 
     CombineArgs ca;
     ca.stop = stop;
@@ -291,6 +319,47 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
                                             step);
     if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
     g_last_launches = 4;
+    return DG_OK;
+}
+
+dg_status dg_profile_enable(int max_records) {
+    if (max_records < 1) return DG_EINVAL;
+    profile_release();
+    g_prof.start.resize(max_records);
+    g_prof.stop.resize(max_records);
+    for (int i = 0; i < max_records; ++i) {
+        if (cudaEventCreate(&g_prof.start[i]) != cudaSuccess || cudaEventCreate(&g_prof.stop[i]) != cudaSuccess) {
+            g_prof.start.resize(i);
+            g_prof.stop.resize(i);
+            profile_release();
+            return DG_ECUDA;
+        }
+    }
+    g_prof.max_records = max_records;
+    g_prof.used = 0;
+    g_prof.on = true;
+    return DG_OK;
+}
+
+dg_status dg_profile_collect(int* n_records, float* mean_ms, float* total_ms) {
+    float total = 0.f;
+    const int n = g_prof.used;
+    for (int i = 0; i < n; ++i) {
+        if (cudaEventSynchronize(g_prof.stop[i]) != cudaSuccess) {
+            profile_release();
+            return DG_ECUDA;
+        }
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, g_prof.start[i], g_prof.stop[i]) != cudaSuccess) {
+            profile_release();
+            return DG_ECUDA;
+        }
+        total += ms;
+    }
+    if (n_records) *n_records = n;
+    if (mean_ms) *mean_ms = n ? total / n : 0.f;
+    if (total_ms) *total_ms = total;
+    profile_release();
     return DG_OK;
 }
 

@@ -100,10 +100,43 @@ inline Layout make_layout(const Plan& pl) {
     return L;
 }
 
-// Units of work: (position tile, vocabulary block) pairs numbered tile-major;
-// group g owns the contiguous range [unit_begin(g), unit_begin(g+1)).
-__host__ __device__ inline long long unit_begin(int g, long long U, int n_groups) {
-    return (static_cast<long long>(g) * U) / n_groups;
+// Work schedule of the fused kernel.  Each position tile's vocabulary blocks are
+// split into k contiguous ranges; the n_pt * k pieces are numbered range-major
+// (pi = j * n_pt + pt) and dealt round-robin to the groups (group pi % n_groups,
+// round pi / n_groups).  Groups working in the same round therefore stream the
+// same vocabulary rows for different tiles at the same time, so the rows are
+// fetched from DRAM once and shared through L2, and every group gets the same
+// number of pieces.  k = n_groups / gcd(n_pt, n_groups) balances exactly; when
+// that would give a group more than kMaxPieces pieces, whole tiles are dealt
+// instead (k = 1).
+constexpr int kMaxPieces = 64;
+
+__host__ __device__ inline int ranges_per_tile(int n_pt, int n_groups) {
+    int a = n_pt, b = n_groups;
+    while (b) {
+        const int t = a % b;
+        a = b;
+        b = t;
+    }
+    const int k = n_groups / a;
+    return (static_cast<long long>(n_pt) * k + n_groups - 1) / n_groups > kMaxPieces ? 1 : k;
+}
+
+__host__ __device__ inline int pieces_per_group(int n_pt, int n_groups) {
+    const int k = ranges_per_tile(n_pt, n_groups);
+    return static_cast<int>((static_cast<long long>(n_pt) * k + n_groups - 1) / n_groups);
+}
+
+// Piece of group g in round j: its position tile and block range [tb, te) (possibly empty).
+__host__ __device__ inline bool piece_of(int g, int j, int n_groups, int n_pt, int T, int& pt, int& tb, int& te) {
+    const int k = ranges_per_tile(n_pt, n_groups);
+    const long long pi = static_cast<long long>(j) * n_groups + g;
+    if (pi >= static_cast<long long>(n_pt) * k) return false;
+    const int jj = static_cast<int>(pi / n_pt);
+    pt = static_cast<int>(pi % n_pt);
+    tb = static_cast<int>(static_cast<long long>(jj) * T / k);
+    te = static_cast<int>(static_cast<long long>(jj + 1) * T / k);
+    return te > tb;
 }
 
 // Offsets of the four per-group counters (uint32 words).

@@ -23,9 +23,10 @@
 //  * Each CTA keeps exact per-row partial statistics of its own tiles relative
 //    to the shared reference: l = sum e, u = sum e (z - m_ref), and the best raw
 //    logit with its smallest vocabulary index.
-//  * A group's contiguous range of (position tile, block) units is split at tile
-//    boundaries into segments; each segment ends with O and the statistics
-//    written as a partial, merged by dg_combine_kernel.
+//  * Work is dealt in pieces (a range of blocks of one position tile) so that
+//    groups in the same round stream the same vocabulary rows for different
+//    tiles (rows come from DRAM once and are shared through L2); each piece ends
+//    with O and the statistics written as a partial, merged by dg_combine_kernel.
 //
 // Roles inside a CTA (256 threads): warp 0 issues TMA loads into a 4-stage ring
 // of 48 KB stages; warp 1 allocates TMEM and issues UMMAs; warps 4-7 (one TMEM
@@ -49,6 +50,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 0;             // logits tile columns [0, 256)
 constexpr uint32_t kTmemO = 256;           // self-conditioning slice columns [256, 256 + slice)
 constexpr int kSoftmaxWarp0 = 4;
+constexpr int kMaxSlotsPerTile = 256;      // >= ranges per tile (at most the group count, <= SM count)
 
 // error codes recorded in the workspace error word
 enum : int {
@@ -105,32 +107,19 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
     tmem_st16(taddr + 16, b);
 }
 
-// The contiguous unit range of one group, split into segments at tile boundaries.
+// The pieces of one group, in round order (see piece_of).
 struct Schedule {
-    long long u0, u1;
-    int T;
-    int pt0;
-    int nseg;
-    __device__ void init(int g, int n_groups, int n_pt, int steps_per_tile) {
+    int g, n_groups, n_pt, T, nseg;
+    __device__ void init(int g_, int n_groups_, int n_pt_, int steps_per_tile) {
+        g = g_;
+        n_groups = n_groups_;
+        n_pt = n_pt_;
         T = steps_per_tile;
-        const long long U = static_cast<long long>(n_pt) * T;
-        u0 = unit_begin(g, U, n_groups);
-        u1 = unit_begin(g + 1, U, n_groups);
-        if (u1 > u0) {
-            pt0 = static_cast<int>(u0 / T);
-            nseg = static_cast<int>((u1 - 1) / T) - pt0 + 1;
-        } else {
-            pt0 = 0;
-            nseg = 0;
-        }
+        nseg = n_pt > 0 ? pieces_per_group(n_pt, n_groups) : 0;
     }
-    __device__ void seg(int j, int& pt, int& tb, int& te) const {
-        pt = pt0 + j;
-        const long long base = static_cast<long long>(pt) * T;
-        const long long lo = u0 > base ? u0 : base;
-        const long long hi = u1 < base + T ? u1 : base + T;
-        tb = static_cast<int>(lo - base);
-        te = static_cast<int>(hi - base);
+    // false for an empty piece (every role skips it the same way)
+    __device__ bool seg(int j, int& pt, int& tb, int& te) const {
+        return piece_of(g, j, n_groups, n_pt, T, pt, tb, te);
     }
 };
 
@@ -243,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
             int k = 0;
             for (int j = 0; j < sch.nseg && ok; ++j) {
                 int pt, tb, te;
-                sch.seg(j, pt, tb, te);
+                if (!sch.seg(j, pt, tb, te)) continue;
                 const int row0 = row0_of(pt);
                 for (int t = tb; t < te && ok; ++t, ++k) {
                     if (sub_valid(t, r)) {
@@ -316,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
             int k = 0;
             for (int j = 0; j < sch.nseg && ok; ++j) {
                 int pt, tb, te;
-                sch.seg(j, pt, tb, te);
+                if (!sch.seg(j, pt, tb, te)) continue;
                 for (int t = tb; t < te && ok; ++t, ++k) {
                     if (k > 0 && !mbar_wait(&s_free, (k - 1) & 1, &abort_flag, a.err, kErrMmaSFree)) {
                         ok = false;
@@ -368,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
         // together and never strand each other at a barrier.
         for (int j = 0; j < sch.nseg && ok; ++j) {
             int pt, tb, te;
-            sch.seg(j, pt, tb, te);
+            if (!sch.seg(j, pt, tb, te)) continue;
             float m_ref = -INFINITY, l = 0.f, u = 0.f, best = -INFINITY;
             int best_idx = -1;
             for (int t = tb; t < te; ++t, ++k) {
@@ -520,8 +509,8 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
 //   sc = sum_s 2^(m_s-M) O_s / L.
 // Block 0 also clears the fused kernel's group counters for its next launch.
 __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
-    __shared__ float sh_w[64];
-    __shared__ int sh_slot[64];
+    __shared__ float sh_w[kMaxSlotsPerTile];
+    __shared__ int sh_slot[kMaxSlotsPerTile];
     __shared__ int n_slots_s;
     __shared__ float sh_L;
     __shared__ int sh_active_rank;
@@ -547,19 +536,21 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
     const int pt = 2 * sh_active_rank + ((n % kCanvas) >= kTileM ? 1 : 0);
     const int row = n % kTileM;
     const int T = a.steps_per_tile;
-    const long long U = static_cast<long long>(2 * n_active) * T;
 
     if (tid < 32) {
         // warp 0: merge statistics over (slot, rank) entries
-        const long long lo = static_cast<long long>(pt) * T, hi = lo + T;
         float M = -INFINITY;
         int ns = 0;
         if (tid == 0) {
-            for (int gg = 0; gg < a.n_groups; ++gg) {
-                const long long u0 = unit_begin(gg, U, a.n_groups), u1 = unit_begin(gg + 1, U, a.n_groups);
-                if (u1 <= u0 || u1 <= lo || u0 >= hi) continue;
-                const int slot = gg * a.max_seg + (pt - static_cast<int>(u0 / T));
-                if (ns < 64) sh_slot[ns++] = slot;
+            const int n_pt = 2 * n_active;
+            const int k = ranges_per_tile(n_pt, a.n_groups);
+            for (int jj = 0; jj < k; ++jj) {
+                const int tb = static_cast<int>(static_cast<long long>(jj) * T / k);
+                const int te = static_cast<int>(static_cast<long long>(jj + 1) * T / k);
+                if (te <= tb) continue;
+                const long long pi = static_cast<long long>(jj) * n_pt + pt;
+                const int gg = static_cast<int>(pi % a.n_groups), round = static_cast<int>(pi / a.n_groups);
+                if (ns < kMaxSlotsPerTile) sh_slot[ns++] = gg * a.max_seg + round;
             }
             n_slots_s = ns;
         }

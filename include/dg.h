@@ -155,6 +155,18 @@ const char* dg_status_string(dg_status s);
 /* Number of kernel launches the last dg_denoise_step on this thread issued. */
 int dg_last_launch_count(void);
 
+/*
+ * Measurement support.  dg_profile_enable(max_records) makes each following
+ * dg_denoise_step on this host thread record a CUDA event pair around its fused
+ * kernel launch, on the caller's stream (events are created here, on the
+ * current device; at most max_records pairs).  dg_profile_collect waits for the
+ * recorded events, returns how many fused launches were recorded and their mean
+ * and total duration in milliseconds, then disables recording and destroys the
+ * events.  Either pointer may be NULL.
+ */
+dg_status dg_profile_enable(int max_records);
+dg_status dg_profile_collect(int* n_records, float* mean_ms, float* total_ms);
+
 /* Column-slice group size and group count the fused kernel uses for p on the current device. */
 dg_status dg_plan(const dg_params* p, int* group, int* n_groups, int* slice_cols);
 

@@ -173,29 +173,36 @@ def denoise_step(h_u16, W_u16, E_u16, T, bound, seeds, s, vocab, canvas_len=256,
 
 
 # ------------------------------------------------------------ large vocabularies
-def logits_chunked(h, W_u16, T, chunk=16384):
-    """z = (h W^T) / T in float64, widening W chunk by chunk (memory only: same arithmetic as ``logits``)."""
+def _widen(block):
+    """bf16 bit patterns are widened to float64; float64 input is used as it is."""
+    return block if block.dtype == np.float64 else bf16_to_f64(block)
+
+
+def logits_chunked(h, W, T, chunk=16384):
+    """z = (h W^T) / T in float64, W (bf16 bits or float64) taken chunk by chunk (memory only)."""
     h = np.asarray(h, np.float64)
-    V = W_u16.shape[0]
+    V = W.shape[0]
     z = np.empty((h.shape[0], V))
     for v0 in range(0, V, chunk):
         v1 = min(V, v0 + chunk)
-        z[:, v0:v1] = (h @ bf16_to_f64(W_u16[v0:v1]).T) / float(T)
+        z[:, v0:v1] = (h @ _widen(W[v0:v1]).T) / float(T)
     return z
 
 
-def self_conditioning_chunked(p, E_u16, chunk=16384):
-    """sc = p E in float64, widening E chunk by chunk (memory only)."""
-    V, d = E_u16.shape
+def self_conditioning_chunked(p, E, chunk=16384):
+    """sc = p E in float64, E (bf16 bits or float64) taken chunk by chunk (memory only)."""
+    V, d = E.shape
     sc = np.zeros((p.shape[0], d))
     for v0 in range(0, V, chunk):
         v1 = min(V, v0 + chunk)
-        sc += p[:, v0:v1] @ bf16_to_f64(E_u16[v0:v1])
+        sc += p[:, v0:v1] @ _widen(E[v0:v1])
     return sc
 
 
 def step_rows(h_u16, W_u16, E_u16, T, bound, seed, s, c, positions, vocab, want_selfcond=True):
     """One step for selected positions of one canvas (rows of h_u16 are those positions).
+
+    W_u16 / E_u16 may be bf16 bit patterns or their exact float64 widening.
 
     positions: index of each row within its canvas (for the re-noise draw).
     Returns dict with H, argmax, lse, top2gap, tokens, accept, selfcond.

@@ -279,3 +279,18 @@ def test_pins_catch_planted_mistakes(monkeypatch):
         assert any(abs(st["H"][i] - ref[i][0]) > 1e-9 for i in range(len(ref)))
     zt = np.zeros((1, 8))
     assert last_index(zt)["argmax"][0] != 0
+
+
+def test_chunked_forms_equal_direct():
+    """The chunked helpers only change memory use: same values as the direct forms."""
+    V, d = 1000, 24
+    W = _rand_bf16((V, d), 0.3, 70)
+    E = _rand_bf16((V, d), 0.3, 71)
+    h = stage.bf16_to_f64(_rand_bf16((7, d), 1.0, 72))
+    z = stage.logits(h, stage.bf16_to_f64(W), 0.6)
+    for Win in (W, stage.bf16_to_f64(W)):
+        zc = stage.logits_chunked(h, Win, 0.6, chunk=97)
+        assert np.array_equal(zc, z)
+    p = stage.distribution_stats(z)["p"]
+    sc = stage.self_conditioning(p, stage.bf16_to_f64(E))
+    assert np.allclose(stage.self_conditioning_chunked(p, E, chunk=97), sc, rtol=1e-13, atol=1e-16)
