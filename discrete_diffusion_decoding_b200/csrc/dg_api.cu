@@ -16,7 +16,7 @@ using namespace dg;
 
 namespace {
 
-constexpr int kFusedSmem = 4 * 48 * 1024 + 1024 + 4 * kMaxCanvas;
+constexpr int kFusedSmem = 6 * 32 * 1024 + 1024 + 4 * kMaxCanvas;
 thread_local int g_last_launches = 0;
 
 // Event pairs recorded around fused-kernel launches while profiling is enabled.
@@ -62,6 +62,43 @@ int device_sm_count() {
     return sms;
 }
 
+bool fused_attr_set() {
+    static std::once_flag once;
+    static cudaError_t err = cudaSuccess;
+    std::call_once(once, [] {
+        err = cudaFuncSetAttribute(dg_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem);
+    });
+    return err == cudaSuccess;
+}
+
+// How many CTA pairs of the fused kernel can be resident at once on the current
+// device (a pair is a cluster of two CTAs, one CTA per SM).
+int resident_pairs() {
+    static int cache[64];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev] > 0) return cache[dev];
+    if (!fused_attr_set()) return -1;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(2 * 64);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kFusedSmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, dg_fused_kernel, &cfg) != cudaSuccess || n <= 0) return -1;
+    cache[dev] = n;
+    return n;
+}
+
 bool params_ok(const dg_params* p) {
     if (!p) return false;
     if (p->n_canvas < 1 || p->n_canvas > kMaxCanvas) return false;
@@ -75,22 +112,24 @@ bool params_ok(const dg_params* p) {
 }
 
 // Returns DG_OK and fills `pl`, or the reason the shape is not handled.
-dg_status make_plan(const dg_params* p, int sms, Plan* pl) {
+// `pairs` is the number of CTA pairs resident at once.
+dg_status make_plan(const dg_params* p, int pairs, Plan* pl) {
     if (!params_ok(p)) return DG_EINVAL;
     int slice = 0;
     if (p->group > 0) {
         if (p->hidden % p->group != 0) return DG_EUNSUPPORTED;
         slice = p->hidden / p->group;
-        if (slice % 64 != 0 || slice > kMaxSlice) return DG_EUNSUPPORTED;
+        if (slice % 128 != 0 || slice > kMaxSlice) return DG_EUNSUPPORTED;
     } else {
-        for (int s = kMaxSlice; s >= 64; s -= 64)
+        for (int s = kMaxSlice; s >= 128; s -= 128)
             if (p->hidden % s == 0) {
                 slice = s;
                 break;
             }
+        if (slice == 0) return DG_EUNSUPPORTED;
     }
     const int G = p->hidden / slice;
-    if (sms < G) return DG_EUNSUPPORTED;
+    if (pairs < G) return DG_EUNSUPPORTED;
     Plan q{};
     q.C = p->n_canvas;
     q.N = p->n_canvas * kCanvas;
@@ -98,12 +137,12 @@ dg_status make_plan(const dg_params* p, int sms, Plan* pl) {
     q.d = p->hidden;
     q.group = G;
     q.slice = slice;
-    q.n_groups = sms / G;
+    q.n_groups = pairs / G;
     q.steps_per_tile = (p->vocab + G * kBV - 1) / (G * kBV);
-    // partial slots per group: the most pieces any active-tile count can give a group
+    // partial slots per group: the most pieces any active-canvas count can give a group
     q.max_seg = 1;
-    for (int n_pt = 2; n_pt <= 2 * q.C; n_pt += 2) {
-        const int pg = pieces_per_group(n_pt, q.n_groups);
+    for (int n_ct = 1; n_ct <= q.C; ++n_ct) {
+        const int pg = pieces_per_group(n_ct, q.n_groups);
         if (pg > q.max_seg) q.max_seg = pg;
     }
     q.n_slots = q.n_groups * q.max_seg;
@@ -176,10 +215,10 @@ const char* dg_status_string(dg_status s) {
 int dg_last_launch_count(void) { return g_last_launches; }
 
 dg_status dg_plan(const dg_params* p, int* group, int* n_groups, int* slice_cols) {
-    const int sms = device_sm_count();
-    if (sms <= 0) return DG_ECUDA;
+    const int pairs = resident_pairs();
+    if (pairs <= 0) return DG_ECUDA;
     Plan pl;
-    dg_status st = make_plan(p, sms, &pl);
+    dg_status st = make_plan(p, pairs, &pl);
     if (st != DG_OK) return st;
     if (group) *group = pl.group;
     if (n_groups) *n_groups = pl.n_groups;
@@ -188,20 +227,20 @@ dg_status dg_plan(const dg_params* p, int* group, int* n_groups, int* slice_cols
 }
 
 size_t dg_workspace_size(const dg_params* p) {
-    const int sms = device_sm_count();
-    if (sms <= 0) return 0;
+    const int pairs = resident_pairs();
+    if (pairs <= 0) return 0;
     Plan pl;
-    if (make_plan(p, sms, &pl) != DG_OK) return 0;
+    if (make_plan(p, pairs, &pl) != DG_OK) return 0;
     return make_layout(pl).total;
 }
 
 dg_status dg_canvas_init(const dg_params* p, const uint64_t* seeds_dev, int32_t* tokens_dev, void* workspace_dev,
                          size_t workspace_bytes, void* stream) {
     g_last_launches = 0;
-    const int sms = device_sm_count();
-    if (sms <= 0) return DG_ECUDA;
+    const int pairs = resident_pairs();
+    if (pairs <= 0) return DG_ECUDA;
     Plan pl;
-    dg_status st = make_plan(p, sms, &pl);
+    dg_status st = make_plan(p, pairs, &pl);
     if (st != DG_OK) return st;
     if (!seeds_dev || !tokens_dev || !workspace_dev) return DG_EINVAL;
     const Layout L = make_layout(pl);
@@ -223,10 +262,10 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
                           uint8_t* accept_dev, float* lse_dev, float* selfcond_dev, void* workspace_dev,
                           size_t workspace_bytes, void* stream) {
     g_last_launches = 0;
-    const int sms = device_sm_count();
-    if (sms <= 0) return DG_ECUDA;
+    const int pairs = resident_pairs();
+    if (pairs <= 0) return DG_ECUDA;
     Plan pl;
-    dg_status st = make_plan(p, sms, &pl);
+    dg_status st = make_plan(p, pairs, &pl);
     if (st != DG_OK) return st;
     if (step < 1 || step > p->max_steps) return DG_EINVAL;
     if (!h_dev || !W_dev || !E_dev || !seeds_dev || !tokens_dev || !entropy_dev || !argmax_dev || !accept_dev ||
@@ -238,18 +277,14 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
     if (workspace_bytes < L.total) return DG_ENOMEM;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(dg_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem);
-    });
-    if (attr_err != cudaSuccess) return DG_ECUDA;
+    if (!fused_attr_set()) return DG_ECUDA;
 
     const float T = dg_temperature(p, step);
     FusedArgs fa;
     std::memset(&fa, 0, sizeof(fa));
-    const uint64_t prow_total = static_cast<uint64_t>(pl.n_groups) * 2 * pl.group * kTileM;
-    if (!encode_2d(&fa.map_h, h_dev, pl.N, pl.d, 64, kTileM) || !encode_2d(&fa.map_w, W_dev, pl.V, pl.d, 64, kBV) ||
+    const uint64_t prow_total = static_cast<uint64_t>(pl.n_groups) * 2 * pl.group * kCanvas;
+    if (!encode_2d(&fa.map_h, h_dev, pl.N, pl.d, 64, kTileM) ||
+        !encode_2d(&fa.map_w, W_dev, pl.V, pl.d, 64, kBV / 2) ||
         !encode_2d(&fa.map_e, E_dev, pl.V, pl.d, 64, kVChunk) ||
         !encode_2d(&fa.map_p, at<void>(workspace_dev, L.pbuf), prow_total, kBV, 64, kTileM))
         return DG_ECUDA;
@@ -274,13 +309,15 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
 
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(pl.n_groups * pl.group);
+    cfg.gridDim = dim3(2 * pl.n_groups * pl.group);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kFusedSmem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
+    attr[0].id = cudaLaunchAttributeClusterDimension;   // CTA pairs
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const bool prof = g_prof.on && g_prof.used < g_prof.max_records;
@@ -365,10 +402,10 @@ dg_status dg_profile_collect(int* n_records, float* mean_ms, float* total_ms) {
 
 dg_status dg_stop_check(const dg_params* p, void* workspace_dev, size_t workspace_bytes, int32_t* stop_flags_host,
                         int32_t* stable_host, int* n_stopped_host, void* stream) {
-    const int sms = device_sm_count();
-    if (sms <= 0) return DG_ECUDA;
+    const int pairs = resident_pairs();
+    if (pairs <= 0) return DG_ECUDA;
     Plan pl;
-    dg_status st = make_plan(p, sms, &pl);
+    dg_status st = make_plan(p, pairs, &pl);
     if (st != DG_OK) return st;
     if (!workspace_dev) return DG_EINVAL;
     const Layout L = make_layout(pl);
@@ -400,10 +437,10 @@ dg_status dg_stub_hidden(const dg_params* p, int step, float gain, float noise, 
                          const void* E_dev, const int32_t* tokens_dev, void* h_dev, void* workspace_dev,
                          size_t workspace_bytes, void* stream) {
     g_last_launches = 0;
-    const int sms = device_sm_count();
-    if (sms <= 0) return DG_ECUDA;
+    const int pairs = resident_pairs();
+    if (pairs <= 0) return DG_ECUDA;
     Plan pl;
-    dg_status st = make_plan(p, sms, &pl);
+    dg_status st = make_plan(p, pairs, &pl);
     if (st != DG_OK) return st;
     if (step < 1 || step > p->max_steps) return DG_EINVAL;
     if (!seeds_dev || !E_dev || !tokens_dev || !h_dev || !workspace_dev) return DG_EINVAL;
@@ -414,7 +451,8 @@ dg_status dg_stub_hidden(const dg_params* p, int step, float gain, float noise, 
     const float a_s = static_cast<float>(static_cast<double>(step) / p->max_steps);
     const long long total = static_cast<long long>(pl.N) * (pl.d / 4);
     long long blocks = (total + 255) / 256;
-    if (blocks > static_cast<long long>(sms) * 16) blocks = static_cast<long long>(sms) * 16;
+    const long long cap = static_cast<long long>(device_sm_count()) * 16;
+    if (cap > 0 && blocks > cap) blocks = cap;
     dg_stub_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(
         seeds_dev, static_cast<const __nv_bfloat16*>(E_dev), tokens_dev, at<int32_t>(workspace_dev, L.stop),
         static_cast<__nv_bfloat16*>(h_dev), a_s, gain, noise, step, pl.d, pl.V, pl.N);

@@ -15,7 +15,7 @@ constexpr int kTileM = 128;       // positions per tile (UMMA M)
 constexpr int kBV = 256;          // vocabulary rows per logits tile (UMMA N)
 constexpr int kKChunk = 64;       // hidden columns per pipeline stage of the logits GEMM
 constexpr int kVChunk = 64;       // vocabulary rows per pipeline stage of the self-conditioning GEMM
-constexpr int kMaxSlice = 256;    // widest self-conditioning column slice one CTA keeps in TMEM
+constexpr int kMaxSlice = 256;    // widest self-conditioning column slice a CTA pair keeps in TMEM
 constexpr int kMaxCanvas = 1024;  // canvases per call (the fused kernel keeps the active list in shared memory)
 constexpr int kThreads = 256;     // threads of the fused kernel
 constexpr float kLazyRescale = 8.0f;  // log2 units the shared reference may lag the running max
@@ -57,10 +57,10 @@ enum : uint32_t { kTagInit = 0, kTagRenoise = 1, kTagStubTarget = 2, kTagStubNoi
 // ------------------------------------------------------------------ plan and layout
 struct Plan {
     int C, N, V, d;
-    int group;        // G: CTAs sharing one logits tile stream, each owning d/G columns
+    int group;        // G: CTA pairs sharing one logits tile stream, each pair owning d/G columns
     int slice;        // d / G
-    int n_groups;     // groups resident at once (grid = n_groups * G CTAs)
-    int steps_per_tile;  // vocabulary blocks of G * kBV rows per position tile
+    int n_groups;     // groups resident at once (grid = n_groups * G pairs = 2 n_groups G CTAs)
+    int steps_per_tile;  // vocabulary blocks of G * kBV rows per canvas
     int max_seg;      // partial slots per group
     int n_slots;      // n_groups * max_seg
 };
@@ -68,11 +68,11 @@ struct Plan {
 struct Layout {
     size_t prev_argmax, stable, stop, err;        // per-canvas state
     size_t counters;                              // [n_groups][4] uint32, 128 B apart
-    size_t rowmax;                                // [n_groups][2][G][128] float
-    size_t pbuf;                                  // [n_groups][2][G][128][kBV] bf16
-    size_t stats;                                 // [n_slots][G][128] float4 {m, l, u, best}
-    size_t stat_idx;                              // [n_slots][G][128] int32
-    size_t opart;                                 // [n_slots][128][d] float
+    size_t rowmax;                                // [n_groups][2][G][256] float
+    size_t pbuf;                                  // [n_groups][2][G][256][kBV] bf16
+    size_t stats;                                 // [n_slots][G][256] float4 {m, l, u, best}
+    size_t stat_idx;                              // [n_slots][G][256] int32
+    size_t opart;                                 // [n_slots][256][d] float
     size_t total;
 };
 
@@ -91,11 +91,11 @@ inline Layout make_layout(const Plan& pl) {
     L.stop = take(sizeof(int32_t) * pl.C);
     L.err = take(sizeof(int32_t) * 4);
     L.counters = take(static_cast<size_t>(128) * 4 * pl.n_groups);
-    L.rowmax = take(sizeof(float) * pl.n_groups * 2 * pl.group * kTileM);
-    L.pbuf = take(static_cast<size_t>(2) * pl.n_groups * 2 * pl.group * kTileM * kBV);
-    L.stats = take(sizeof(float) * 4 * pl.n_slots * pl.group * kTileM);
-    L.stat_idx = take(sizeof(int32_t) * pl.n_slots * pl.group * kTileM);
-    L.opart = take(sizeof(float) * static_cast<size_t>(pl.n_slots) * kTileM * pl.d);
+    L.rowmax = take(sizeof(float) * pl.n_groups * 2 * pl.group * kCanvas);
+    L.pbuf = take(static_cast<size_t>(2) * pl.n_groups * 2 * pl.group * kCanvas * kBV);
+    L.stats = take(sizeof(float) * 4 * static_cast<size_t>(pl.n_slots) * pl.group * kCanvas);
+    L.stat_idx = take(sizeof(int32_t) * static_cast<size_t>(pl.n_slots) * pl.group * kCanvas);
+    L.opart = take(sizeof(float) * static_cast<size_t>(pl.n_slots) * kCanvas * pl.d);
     L.total = o;
     return L;
 }

@@ -7,31 +7,36 @@
 // steps 3-5 and the entropy criteria):
 //   z = h W^T / T;  p = softmax(z);  H = LSE - sum p z;  a = argmax z;  sc = p E.
 //
-// Work decomposition (sm_100a, one CTA per SM, persistent, cooperative launch):
-//  * A position tile is 128 canvas positions (UMMA M = 128).
-//  * A group of G CTAs streams the vocabulary in blocks of G x 256 rows.  In a
-//    block, CTA r computes the 256-wide logits tile of vocabulary sub-tile r over
-//    the full hidden width (TMA -> SMEM -> tcgen05.mma -> TMEM), and owns columns
-//    [r*d/G, (r+1)*d/G) of the self-conditioning accumulator O (fp32, in TMEM).
-//  * The G CTAs agree on a per-row reference maximum for the block (row maxima
-//    exchanged through L2 with release/acquire counters), so every CTA turns its
-//    logits tile into P = 2^(z*log2e - m_ref) in bf16 against the same reference,
-//    publishes P to an L2-resident scratch tile, and accumulates
-//    O[:, slice] += P_q E[q-rows, slice] for all G tiles q of the block (second
-//    tcgen05 GEMM, E as an MN-major operand).  The reference only moves when the
-//    running maximum exceeds it by 8 (log2 units), and then O is rescaled in TMEM.
+// Work decomposition (sm_100a, persistent grid of CTA pairs, one CTA per SM):
+//  * A CTA pair (cluster of 2, cta_group::2 UMMA) owns one 256-position canvas:
+//    CTA p holds positions [128p, 128p+128) (UMMA M = 256 split across the pair).
+//  * A group of G pairs streams the vocabulary in blocks of G x 256 rows.  In a
+//    block, pair r computes the 256 x 256 logits tile of vocabulary sub-tile r over
+//    the full hidden width (each CTA loads its own h rows and half of the 256 W
+//    rows; TMA -> SMEM -> tcgen05.mma -> TMEM), and owns columns
+//    [r d/G, (r+1) d/G) of the self-conditioning accumulator O (fp32, TMEM).
+//  * The CTAs of a group agree on a per-row reference maximum for the block (row
+//    maxima exchanged through L2 with release/acquire counters), so every CTA
+//    turns its logits into P = 2^(z log2e - m_ref) in bf16 against the same
+//    reference, publishes P to an L2-resident scratch tile, and the pair
+//    accumulates O[:, slice] += P_q E[q-rows, slice] for all G tiles q of the
+//    block (second pair UMMA, E as an MN-major operand split by columns).  The
+//    reference only moves when the running maximum exceeds it by 8 (log2 units),
+//    and then O is rescaled in TMEM.
 //  * Each CTA keeps exact per-row partial statistics of its own tiles relative
 //    to the shared reference: l = sum e, u = sum e (z - m_ref), and the best raw
 //    logit with its smallest vocabulary index.
-//  * Work is dealt in pieces (a range of blocks of one position tile) so that
-//    groups in the same round stream the same vocabulary rows for different
-//    tiles (rows come from DRAM once and are shared through L2); each piece ends
-//    with O and the statistics written as a partial, merged by dg_combine_kernel.
+//  * Work is dealt in pieces (a range of blocks of one canvas) so that groups in
+//    the same round stream the same vocabulary rows for different canvases (rows
+//    come from DRAM once and are shared through L2); each piece ends with O and
+//    the statistics written as a partial, merged by dg_combine_kernel.
 //
-// Roles inside a CTA (256 threads): warp 0 issues TMA loads into a 4-stage ring
-// of 48 KB stages; warp 1 allocates TMEM and issues UMMAs; warps 4-7 (one TMEM
-// lane quarter each, thread = position row) do the softmax, publish P and run
-// the epilogue.  Every wait is bounded (see dg_sm100.cuh).
+// Roles inside a CTA (256 threads): warp 0 issues TMA loads into a 6-stage ring
+// of 32 KB stages (both CTAs of a pair load; completion is counted on the
+// leader's barriers); warp 1 allocates TMEM and, in the leader CTA, issues the
+// pair UMMAs; warps 4-7 (one TMEM lane quarter each, thread = position row) do
+// the softmax, publish P and run the epilogue.  Every wait is bounded (see
+// dg_sm100.cuh).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -44,13 +49,14 @@ namespace dg {
 
 namespace {
 
-constexpr int kStages = 4;
-constexpr int kStageBytes = 48 * 1024;     // S stage: h 16 KB + W 32 KB; O stage: P 16 KB + E 32 KB
+constexpr int kStages = 6;
+constexpr int kStageBytes = 32 * 1024;     // per CTA: A operand 16 KB + B operand half 16 KB
+constexpr int kHalfB = 16 * 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 0;             // logits tile columns [0, 256)
 constexpr uint32_t kTmemO = 256;           // self-conditioning slice columns [256, 256 + slice)
 constexpr int kSoftmaxWarp0 = 4;
-constexpr int kMaxSlotsPerTile = 256;      // >= ranges per tile (at most the group count, <= SM count)
+constexpr int kMaxSlotsPerTile = 256;      // >= ranges per tile (at most the group count)
 
 // error codes recorded in the workspace error word
 enum : int {
@@ -109,17 +115,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 
 // The pieces of one group, in round order (see piece_of).
 struct Schedule {
-    int g, n_groups, n_pt, T, nseg;
-    __device__ void init(int g_, int n_groups_, int n_pt_, int steps_per_tile) {
+    int g, n_groups, n_ct, T, nseg;
+    __device__ void init(int g_, int n_groups_, int n_ct_, int steps_per_tile) {
         g = g_;
         n_groups = n_groups_;
-        n_pt = n_pt_;
+        n_ct = n_ct_;
         T = steps_per_tile;
-        nseg = n_pt > 0 ? pieces_per_group(n_pt, n_groups) : 0;
+        nseg = n_ct > 0 ? pieces_per_group(n_ct, n_groups) : 0;
     }
     // false for an empty piece (every role skips it the same way)
-    __device__ bool seg(int j, int& pt, int& tb, int& te) const {
-        return piece_of(g, j, n_groups, n_pt, T, pt, tb, te);
+    __device__ bool seg(int j, int& ct, int& tb, int& te) const {
+        return piece_of(g, j, n_groups, n_ct, T, ct, tb, te);
     }
 };
 
@@ -141,18 +147,21 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const int G = a.G;
-    const int g = blockIdx.x / G;
-    const int r = blockIdx.x % G;
+    const uint32_t prank = cluster_ctarank();        // 0 = pair leader (issues the UMMAs)
+    const bool leader = prank == 0;
+    const int pair = blockIdx.x >> 1;
+    const int g = pair / G;
+    const int r = pair % G;
     const int d0 = r * a.slice;
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&full_bar[i], 1);
-            mbar_init(&empty_bar[i], 1);
+            mbar_init(&full_bar[i], 1);      // leader: one expect_tx arrival per use, bytes of both CTAs
+            mbar_init(&empty_bar[i], 1);     // one multicast commit per use
         }
         mbar_init(&s_full, 1);
-        mbar_init(&s_free, 1);
-        mbar_init(&o_ready, 1);
+        mbar_init(&s_free, 2);               // leader: softmax of both CTAs
+        mbar_init(&o_ready, 2);              // leader: softmax of both CTAs
         mbar_init(&o_done, 1);
         mbar_init(&drain_bar, 1);
         fence_mbar_init_cluster();
@@ -172,33 +181,35 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
         if (lane == 0) n_active_s = base;
     }
     if (warp == 1) {
-        tmem_alloc(&tmem_base, kTmemCols);
-        tmem_relinquish();
+        tmem_alloc_pair(&tmem_base, kTmemCols);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();        // barriers of both CTAs initialised before any remote arrival
     tc_fence_after();
 
     const uint32_t tmem = tmem_base;
     Schedule sch;
-    sch.init(g, a.n_groups, 2 * n_active_s, a.steps_per_tile);
+    sch.init(g, a.n_groups, n_active_s, a.steps_per_tile);
     auto sub_valid = [&](int t, int q) { return static_cast<long long>(t * G + q) * kBV < a.V; };
     auto vocab0 = [&](int t, int q) { return (t * G + q) * kBV; };
-    auto row0_of = [&](int pt) { return active[pt >> 1] * kCanvas + (pt & 1) * kTileM; };
 
     uint32_t* cnt_rowmax = a.counters + counter_word(g, kCntRowmax);
     uint32_t* cnt_p = a.counters + counter_word(g, kCntP);
     uint32_t* cnt_used = a.counters + counter_word(g, kCntUsed);
-    const int n_ech = a.slice / 64;                 // E boxes per O stage
+    const int n_ech = a.slice / 128;                 // E boxes (64 columns each) per CTA per O stage
     const uint32_t o_stage_bytes = 16384u + static_cast<uint32_t>(n_ech) * 8192u;
+    const int nG2 = 2 * G;                           // CTAs per group
 
     if (warp == 0) {
-        // ===================================================== TMA producer
+        // ===================================================== TMA producer (both CTAs)
         if (lane == 0) {
             tma_prefetch_desc(&a.map_h);
             tma_prefetch_desc(&a.map_w);
             tma_prefetch_desc(&a.map_e);
             tma_prefetch_desc(&a.map_p);
+            // the leader's full barrier of a stage, as a shared::cluster address
+            auto full_leader = [&](int slot) { return smem_addr_in_rank(&full_bar[slot], 0); };
             uint32_t it = 0;
             bool ok = true;
             auto acquire = [&](int& slot) -> bool {
@@ -210,51 +221,53 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                 return true;
             };
             auto emit_o = [&](int k, int t) -> bool {
-                if (!wait_counter(cnt_p, static_cast<uint32_t>(G * (k + 1)), &abort_flag, a.err, kErrProducerP))
+                if (!wait_counter(cnt_p, static_cast<uint32_t>(nG2 * (k + 1)), &abort_flag, a.err, kErrProducerP))
                     return false;
                 fence_async_global();
                 for (int q = 0; q < G; ++q) {
                     if (!sub_valid(t, q)) continue;
-                    const int prow = ((g * 2 + (k & 1)) * G + q) * kTileM;
+                    const int prow = ((g * 2 + (k & 1)) * G + q) * kCanvas + static_cast<int>(prank) * kTileM;
                     for (int c4 = 0; c4 < kBV / kVChunk; ++c4) {
                         int slot;
                         if (!acquire(slot)) return false;
                         uint8_t* st = ring + slot * kStageBytes;
-                        mbar_arrive_expect_tx(&full_bar[slot], o_stage_bytes);
-                        tma_load_2d(st, &a.map_p, &full_bar[slot], c4 * kVChunk, prow);
+                        if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2u * o_stage_bytes);
+                        tma_load_2d_pair(st, &a.map_p, full_leader(slot), c4 * kVChunk, prow);
                         for (int j = 0; j < n_ech; ++j)
-                            tma_load_2d(st + 16384 + j * 8192, &a.map_e, &full_bar[slot], d0 + j * 64,
-                                        vocab0(t, q) + c4 * kVChunk);
+                            tma_load_2d_pair(st + kHalfB + j * 8192, &a.map_e, full_leader(slot),
+                                             d0 + static_cast<int>(prank) * (a.slice / 2) + j * 64,
+                                             vocab0(t, q) + c4 * kVChunk);
                     }
                 }
                 return true;
             };
             int k = 0;
             for (int j = 0; j < sch.nseg && ok; ++j) {
-                int pt, tb, te;
-                if (!sch.seg(j, pt, tb, te)) continue;
-                const int row0 = row0_of(pt);
+                int ct, tb, te;
+                if (!sch.seg(j, ct, tb, te)) continue;
+                const int row0 = active[ct] * kCanvas + static_cast<int>(prank) * kTileM;
                 for (int t = tb; t < te && ok; ++t, ++k) {
                     if (sub_valid(t, r)) {
-                        const int v0 = vocab0(t, r);
+                        const int v0 = vocab0(t, r) + static_cast<int>(prank) * (kBV / 2);
                         for (int kc = 0; kc < a.d / kKChunk; ++kc) {
                             int slot;
                             if (!acquire(slot)) { ok = false; break; }
                             uint8_t* st = ring + slot * kStageBytes;
-                            mbar_arrive_expect_tx(&full_bar[slot], 16384u + 32768u);
-                            tma_load_2d(st, &a.map_h, &full_bar[slot], kc * kKChunk, row0);
-                            tma_load_2d(st + 16384, &a.map_w, &full_bar[slot], kc * kKChunk, v0);
+                            if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2u * kStageBytes);
+                            tma_load_2d_pair(st, &a.map_h, full_leader(slot), kc * kKChunk, row0);
+                            tma_load_2d_pair(st + kHalfB, &a.map_w, full_leader(slot), kc * kKChunk, v0);
                         }
                     }
                     if (ok && t > tb) ok = emit_o(k - 1, t - 1);
                 }
                 if (ok) ok = emit_o(k - 1, te - 1);
             }
-            // drain: every issued load must have landed before the CTA may exit
+            // drain: every issued use of a stage has been released by the leader's
+            // commit, so no load into this CTA is still in flight when it exits
             for (uint32_t u = (it > kStages ? it - kStages : 0); u < it; ++u) {
                 const int slot = static_cast<int>(u % kStages);
-                uint64_t t0 = global_ns();
-                while (!mbar_try_wait(smem_u32(&full_bar[slot]), (u / kStages) & 1)) {
+                const uint64_t t0 = global_ns();
+                while (!mbar_try_wait(smem_u32(&empty_bar[slot]), (u / kStages) & 1)) {
                     if (global_ns() - t0 > DG_WAIT_LIMIT_NS) {
                         atomicCAS(a.err, 0, kErrProducerDrain);
                         break;
@@ -263,10 +276,10 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
             }
         }
     } else if (warp == 1) {
-        // ===================================================== UMMA issuer
-        if (lane == 0) {
-            const uint32_t idesc_s = idesc_bf16_f32(kTileM, kBV, false, false);
-            const uint32_t idesc_o = idesc_bf16_f32(kTileM, a.slice, false, true);
+        // ===================================================== pair UMMA issuer (leader CTA)
+        if (lane == 0 && leader) {
+            const uint32_t idesc_s = idesc_bf16_f32(2 * kTileM, kBV, false, false);
+            const uint32_t idesc_o = idesc_bf16_f32(2 * kTileM, a.slice, false, true);
             uint32_t it = 0;
             bool ok = true;
             auto consume = [&](int& slot) -> bool {
@@ -276,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                 tc_fence_after();
                 return true;
             };
-            // seg_first: block t is the first of its segment, so O starts from zero
+            // seg_first: block t is the first of its piece, so O starts from zero
             auto do_o = [&](int k, int t, bool seg_first) -> bool {
                 if (!mbar_wait(&o_ready, k & 1, &abort_flag, a.err, kErrMmaOReady)) return false;
                 tc_fence_after();
@@ -290,22 +303,22 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
 #pragma unroll
                         for (int kk = 0; kk < kVChunk / 16; ++kk) {
                             const uint64_t ad = smem_desc(st + kk * 32, 16, 1024, kSwizzle128B);
-                            const uint64_t bd = smem_desc(st + 16384 + kk * 2048, 8192, 1024, kSwizzle128B);
-                            umma_ss(tmem + kTmemO, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
+                            const uint64_t bd = smem_desc(st + kHalfB + kk * 2048, 8192, 1024, kSwizzle128B);
+                            umma_ss_pair(tmem + kTmemO, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
                         }
                         first = false;
-                        umma_commit(&empty_bar[slot]);
+                        umma_commit_pair(&empty_bar[slot], 0x3);
                     }
                 }
-                // every P tile of block k has landed in this CTA's shared memory
+                // every P tile of block k has landed in both CTAs' shared memory
                 red_release_add(cnt_used, 1u);
-                umma_commit(&o_done);
+                umma_commit_pair(&o_done, 0x3);
                 return true;
             };
             int k = 0;
             for (int j = 0; j < sch.nseg && ok; ++j) {
-                int pt, tb, te;
-                if (!sch.seg(j, pt, tb, te)) continue;
+                int ct, tb, te;
+                if (!sch.seg(j, ct, tb, te)) continue;
                 for (int t = tb; t < te && ok; ++t, ++k) {
                     if (k > 0 && !mbar_wait(&s_free, (k - 1) & 1, &abort_flag, a.err, kErrMmaSFree)) {
                         ok = false;
@@ -320,23 +333,24 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
 #pragma unroll
                             for (int kk = 0; kk < kKChunk / 16; ++kk) {
                                 const uint64_t ad = smem_desc(st + kk * 32, 16, 1024, kSwizzle128B);
-                                const uint64_t bd = smem_desc(st + 16384 + kk * 32, 16, 1024, kSwizzle128B);
-                                umma_ss(tmem + kTmemS, ad, bd, idesc_s, (kc | kk) != 0 ? 1u : 0u);
+                                const uint64_t bd = smem_desc(st + kHalfB + kk * 32, 16, 1024, kSwizzle128B);
+                                umma_ss_pair(tmem + kTmemS, ad, bd, idesc_s, (kc | kk) != 0 ? 1u : 0u);
                             }
-                            umma_commit(&empty_bar[slot]);
+                            umma_commit_pair(&empty_bar[slot], 0x3);
                         }
                         if (!ok) break;
-                        umma_commit(&s_full);
+                        umma_commit_pair(&s_full, 0x3);
                     } else {
-                        mbar_arrive(&s_full);
+                        mbar_arrive_remote(&s_full, 0);
+                        mbar_arrive_remote(&s_full, 1);
                     }
                     if (t > tb) ok = do_o(k - 1, t - 1, t - 1 == tb);
                 }
                 if (ok) ok = do_o(k - 1, te - 1, te - 1 == tb);
             }
             // drain: all issued UMMAs complete before TMEM is released
-            umma_commit(&drain_bar);
-            uint64_t t0 = global_ns();
+            umma_commit_pair(&drain_bar, 0x1);
+            const uint64_t t0 = global_ns();
             while (!mbar_try_wait(smem_u32(&drain_bar), 0)) {
                 if (global_ns() - t0 > DG_WAIT_LIMIT_NS) {
                     atomicCAS(a.err, 0, kErrMmaDrain);
@@ -346,18 +360,19 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
         }
     } else if (warp >= kSoftmaxWarp0) {
         // ===================================================== softmax / epilogue
-        const int row = (warp - kSoftmaxWarp0) * 32 + lane;
-        const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const bool leader = (tid == kSoftmaxWarp0 * 32);
-        const float c2 = a.scale_log2;
-        bool ok = true;
-        int k = 0;
         // Every bounded wait below is followed by a softmax-warp barrier and a
         // check of the shared abort flag, so the 128 threads always leave
         // together and never strand each other at a barrier.
+        const int row = (warp - kSoftmaxWarp0) * 32 + lane;      // row within this CTA's 128
+        const int crow = static_cast<int>(prank) * kTileM + row; // row within the canvas
+        const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const bool sleader = (tid == kSoftmaxWarp0 * 32);
+        const float c2 = a.scale_log2;
+        bool ok = true;
+        int k = 0;
         for (int j = 0; j < sch.nseg && ok; ++j) {
-            int pt, tb, te;
-            if (!sch.seg(j, pt, tb, te)) continue;
+            int ct, tb, te;
+            if (!sch.seg(j, ct, tb, te)) continue;
             float m_ref = -INFINITY, l = 0.f, u = 0.f, best = -INFINITY;
             int best_idx = -1;
             for (int t = tb; t < te; ++t, ++k) {
@@ -378,14 +393,14 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                         for (int i = 0; i < 32; ++i) smax = fmaxf(smax, __uint_as_float(v[i]));
                     }
                 }
-                float* rm = a.rowmax + static_cast<size_t>((g * 2 + (k & 1)) * G) * kTileM;
-                rm[r * kTileM + row] = smax * c2;
+                float* rm = a.rowmax + static_cast<size_t>((g * 2 + (k & 1)) * G) * kCanvas;
+                rm[r * kCanvas + crow] = smax * c2;
                 __threadfence();
                 softmax_bar();
-                if (leader) {
+                if (sleader) {
                     red_release_add(cnt_rowmax, 1u);
-                    bool w = wait_counter(cnt_rowmax, static_cast<uint32_t>(G * (k + 1)), &abort_flag, a.err,
-                                          kErrSmaxRowmax);
+                    const bool w = wait_counter(cnt_rowmax, static_cast<uint32_t>(nG2 * (k + 1)), &abort_flag,
+                                                a.err, kErrSmaxRowmax);
                     // P buffer (k & 1) was last read for block k-2
                     if (w && k >= 2)
                         wait_counter(cnt_used, static_cast<uint32_t>(G * (k - 1)), &abort_flag, a.err, kErrSmaxUsed);
@@ -393,8 +408,8 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                 softmax_bar();
                 if (abort_flag) { ok = false; break; }
                 float M = -INFINITY;
-                for (int q = 0; q < G; ++q) M = fmaxf(M, __ldcg(rm + q * kTileM + row));
-                // --- lazy shared reference (the same decision in all G CTAs of the group)
+                for (int q = 0; q < G; ++q) M = fmaxf(M, __ldcg(rm + q * kCanvas + crow));
+                // --- lazy shared reference (the same decision in all CTAs holding this row)
                 float alpha = 1.f;
                 if (m_ref == -INFINITY || M > m_ref + kLazyRescale) {
                     if (m_ref != -INFINITY) {
@@ -407,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                 // --- pass 2: probabilities, statistics, argmax, P tile
                 if (valid) {
                     __nv_bfloat16* prow =
-                        a.pbuf + (static_cast<size_t>((g * 2 + (k & 1)) * G + r) * kTileM + row) * kBV;
+                        a.pbuf + (static_cast<size_t>((g * 2 + (k & 1)) * G + r) * kCanvas + crow) * kBV;
                     const int v0 = vocab0(t, r);
 #pragma unroll 1
                     for (int c0 = 0; c0 < kBV; c0 += 32) {
@@ -438,8 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                 if (alpha != 1.f && t > tb) rescale_any = 1;
                 softmax_bar();
                 const bool resc = rescale_any != 0;
-                if (leader) {
-                    mbar_arrive(&s_free);
+                if (sleader) {
+                    mbar_arrive_remote(&s_free, 0);
                     red_release_add(cnt_p, 1u);
                 }
                 // --- O of block k-1 must be complete before block k may accumulate (and be rescaled)
@@ -463,19 +478,19 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                     tc_fence_before();
                 }
                 softmax_bar();
-                if (leader) {
+                if (sleader) {
                     rescale_any = 0;
-                    mbar_arrive(&o_ready);
+                    mbar_arrive_remote(&o_ready, 0);
                 }
             }
             if (!ok) break;
-            // --- segment epilogue: O slice and statistics become a partial
+            // --- piece epilogue: O slice and statistics become a partial
             mbar_wait(&o_done, (k - 1) & 1, &abort_flag, a.err, kErrSmaxODone);
             softmax_bar();
             if (abort_flag) { ok = false; break; }
             tc_fence_after();
             const int slot = g * a.max_seg + j;
-            float* orow = a.opart + (static_cast<size_t>(slot) * kTileM + row) * a.d + d0;
+            float* orow = a.opart + (static_cast<size_t>(slot) * kCanvas + crow) * a.d + d0;
 #pragma unroll 1
             for (int c0 = 0; c0 < a.slice; c0 += 32) {
                 uint32_t v[32];
@@ -487,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                     dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
                                          __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
             }
-            const size_t si = (static_cast<size_t>(slot) * G + r) * kTileM + row;
+            const size_t si = (static_cast<size_t>(slot) * G + r) * kCanvas + crow;
             a.stats[si] = make_float4(m_ref, l, u, best);
             a.stat_idx[si] = best_idx;
             tc_fence_before();
@@ -497,13 +512,14 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
 
     tc_fence_before();
     __syncthreads();
+    cluster_sync_all();        // no CTA leaves while its peer may still signal it
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+    if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
 }
 
 // ---------------------------------------------------------------------------
 // Split-vocabulary combine: one CTA per active position.  Merges the partial
-// statistics of every (segment, rank) covering the position's tile:
+// statistics of every (piece, pair) covering the position's canvas:
 //   M = max m_s;  L = sum_s 2^(m_s-M) sum_r l;  U = sum_s 2^(m_s-M) (sum_r u + (m_s-M) sum_r l)
 //   H = ln L - ln2 * U / L;  LSE = ln2 * (M + log2 L);  argmax = best raw logit, smallest index;
 //   sc = sum_s 2^(m_s-M) O_s / L.
@@ -514,41 +530,44 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
     __shared__ int n_slots_s;
     __shared__ float sh_L;
     __shared__ int sh_active_rank;
+    __shared__ int sh_n_active;
     __shared__ int sh_skip;
 
     const int n = blockIdx.x;               // position row in [0, N)
     const int c = n / kCanvas;
+    const int crow = n % kCanvas;
     const int tid = threadIdx.x;
     if (blockIdx.x == 0) {
         for (int i = tid; i < a.n_groups * 128; i += blockDim.x) a.counters[i] = 0u;
     }
     if (tid == 0) {
         sh_skip = a.stop[c] != 0;
-        // rank of canvas c among the active canvases
-        int rank = 0;
-        for (int q = 0; q < c; ++q) rank += a.stop[q] == 0;
+        int rank = 0, na = 0;
+        for (int q = 0; q < a.C; ++q) {
+            const int act = a.stop[q] == 0;
+            if (q < c) rank += act;
+            na += act;
+        }
         sh_active_rank = rank;
+        sh_n_active = na;
     }
     __syncthreads();
     if (sh_skip) return;
-    int n_active = 0;
-    for (int q = 0; q < a.C; ++q) n_active += a.stop[q] == 0;   // same in every thread
-    const int pt = 2 * sh_active_rank + ((n % kCanvas) >= kTileM ? 1 : 0);
-    const int row = n % kTileM;
+    const int ct = sh_active_rank;
     const int T = a.steps_per_tile;
 
     if (tid < 32) {
-        // warp 0: merge statistics over (slot, rank) entries
+        // warp 0: merge statistics over (slot, pair) entries
         float M = -INFINITY;
         int ns = 0;
         if (tid == 0) {
-            const int n_pt = 2 * n_active;
-            const int k = ranges_per_tile(n_pt, a.n_groups);
+            const int n_ct = sh_n_active;
+            const int k = ranges_per_tile(n_ct, a.n_groups);
             for (int jj = 0; jj < k; ++jj) {
                 const int tb = static_cast<int>(static_cast<long long>(jj) * T / k);
                 const int te = static_cast<int>(static_cast<long long>(jj + 1) * T / k);
                 if (te <= tb) continue;
-                const long long pi = static_cast<long long>(jj) * n_pt + pt;
+                const long long pi = static_cast<long long>(jj) * n_ct + ct;
                 const int gg = static_cast<int>(pi % a.n_groups), round = static_cast<int>(pi / a.n_groups);
                 if (ns < kMaxSlotsPerTile) sh_slot[ns++] = gg * a.max_seg + round;
             }
@@ -556,12 +575,13 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
         }
         __syncwarp();
         ns = n_slots_s;
-        for (int s = 0; s < ns; ++s) M = fmaxf(M, a.stats[(static_cast<size_t>(sh_slot[s]) * a.G) * kTileM + row].x);
+        for (int s = 0; s < ns; ++s)
+            M = fmaxf(M, a.stats[(static_cast<size_t>(sh_slot[s]) * a.G) * kCanvas + crow].x);
         float L = 0.f, Uu = 0.f, best = -INFINITY;
         int bidx = 0x7fffffff;
         for (int e = tid; e < ns * a.G; e += 32) {
             const int s = e / a.G, rr = e % a.G;
-            const size_t si = (static_cast<size_t>(sh_slot[s]) * a.G + rr) * kTileM + row;
+            const size_t si = (static_cast<size_t>(sh_slot[s]) * a.G + rr) * kCanvas + crow;
             const float4 st = a.stats[si];
             const int idx = a.stat_idx[si];
             const float w = exp2f(st.x - M);
@@ -591,7 +611,8 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
             if (a.lse) a.lse[n] = ln2 * (M + log2f(L));
             sh_L = L;
         }
-        for (int s = tid; s < ns; s += 32) sh_w[s] = exp2f(a.stats[(static_cast<size_t>(sh_slot[s]) * a.G) * kTileM + row].x - M);
+        for (int s = tid; s < ns; s += 32)
+            sh_w[s] = exp2f(a.stats[(static_cast<size_t>(sh_slot[s]) * a.G) * kCanvas + crow].x - M);
     }
     __syncthreads();
     if (a.selfcond == nullptr) return;
@@ -600,7 +621,8 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
     for (int col = tid * 4; col < a.d; col += blockDim.x * 4) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int s = 0; s < ns; ++s) {
-            const float4 o = *reinterpret_cast<const float4*>(a.opart + (static_cast<size_t>(sh_slot[s]) * kTileM + row) * a.d + col);
+            const float4 o =
+                *reinterpret_cast<const float4*>(a.opart + (static_cast<size_t>(sh_slot[s]) * kCanvas + crow) * a.d + col);
             const float w = sh_w[s];
             acc.x = fmaf(w, o.x, acc.x);
             acc.y = fmaf(w, o.y, acc.y);

@@ -100,11 +100,10 @@ def test_step_small_tied(dg, kind):
         assert 0 < int(g["accept"].sum()) < C * 256           # both branches of the sampler taken
 
 
-@pytest.mark.parametrize("group,tied,C,V", [(2, True, 2, 8960), (4, False, 2, 8960), (8, True, 3, 4096),
-                                            (1, True, 2, 65536)])
-def test_step_groups_and_segments(dg, group, tied, C, V):
-    """Multi-CTA groups (P exchange, shared reference), tile-spanning segments, ragged blocks."""
-    d = 512 if group > 1 else 256
+@pytest.mark.parametrize("group,tied,C,V,d", [(2, True, 2, 8960, 512), (4, False, 2, 8960, 512),
+                                              (8, True, 3, 4096, 1024), (1, True, 2, 65536, 256)])
+def test_step_groups_and_segments(dg, group, tied, C, V, d):
+    """Multi-pair groups (P exchange, shared reference), multi-block pieces, ragged blocks."""
     W = synth.weights(V, d, seed=1234)
     E = W if tied else synth.weights(V, d, seed=1235)
     h, _ = synth.spiked_hidden(W, C * 256, seed=50 + group, gain_lo=0.5, gain_hi=30.0)
@@ -299,6 +298,8 @@ def test_argument_errors(dg):
         dg.workspace_size(dg.params(1, 4000, 128))            # vocab not a multiple of 256
     with pytest.raises(_abi.DgError):
         dg.workspace_size(dg.params(1, 4096, 100))            # hidden not a multiple of 64
+    with pytest.raises(_abi.DgError):
+        dg.workspace_size(dg.params(1, 4096, 192))            # no column slice of 128 or 256 divides it
     bad = dg.params(1, 4096, 512, group=3)
     with pytest.raises(_abi.DgError) as e:
         dg.plan(bad)
