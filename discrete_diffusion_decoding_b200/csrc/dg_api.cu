@@ -286,7 +286,7 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
     if (!encode_2d(&fa.map_h, h_dev, pl.N, pl.d, 64, kTileM) ||
         !encode_2d(&fa.map_w, W_dev, pl.V, pl.d, 64, kBV / 2) ||
         !encode_2d(&fa.map_e, E_dev, pl.V, pl.d, 64, kVChunk) ||
-        !encode_2d(&fa.map_p, at<void>(workspace_dev, L.pbuf), prow_total, kBV, 64, kTileM))
+        !encode_2d(&fa.map_p, at<void>(workspace_dev, L.pbuf), prow_total, kCanvas, 64, kVChunk))
         return DG_ECUDA;
     int32_t* stop = at<int32_t>(workspace_dev, L.stop);
     fa.stop = stop;

@@ -69,7 +69,7 @@ struct Layout {
     size_t prev_argmax, stable, stop, err;        // per-canvas state
     size_t counters;                              // [n_groups][4] uint32, 128 B apart
     size_t rowmax;                                // [n_groups][2][G][256] float
-    size_t pbuf;                                  // [n_groups][2][G][256][kBV] bf16
+    size_t pbuf;                                  // [n_groups][2][G][kBV vocab][256 rows] bf16 (P^T)
     size_t stats;                                 // [n_slots][G][256] float4 {m, l, u, best}
     size_t stat_idx;                              // [n_slots][G][256] int32
     size_t opart;                                 // [n_slots][256][d] float

@@ -31,12 +31,12 @@
 //    come from DRAM once and are shared through L2); each piece ends with O and
 //    the statistics written as a partial, merged by dg_combine_kernel.
 //
-// Roles inside a CTA (256 threads): warp 0 issues TMA loads into a 6-stage ring
-// of 32 KB stages (both CTAs of a pair load; completion is counted on the
-// leader's barriers); warp 1 allocates TMEM and, in the leader CTA, issues the
-// pair UMMAs; warps 4-7 (one TMEM lane quarter each, thread = position row) do
-// the softmax, publish P and run the epilogue.  Every wait is bounded (see
-// dg_sm100.cuh).
+// Roles inside a CTA (256 threads): warps 0 and 3 issue TMA loads (A and B
+// operands) into a 6-stage ring of 32 KB stages (both CTAs of a pair load;
+// completion is counted on the leader's barriers); warp 1 allocates TMEM and,
+// in the leader CTA, issues the pair UMMAs; warps 4-7 (one TMEM lane quarter
+// each, thread = position row) do the softmax, publish P^T and run the epilogue.
+// Every wait is bounded (see dg_sm100.cuh).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -96,6 +96,22 @@ __device__ bool wait_counter(const uint32_t* ctr, uint32_t target, volatile int*
 }
 
 __device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// 2^x on the SFU (documented PTX ex2.approx; relative error about 2^-22, 2^-inf = +0).
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// 64 consecutive TMEM columns of this thread's lane, two loads in flight per wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&v)[64]) {
+    uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
+    uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
+    tmem_ld32(taddr, lo);
+    tmem_ld32(taddr + 32, hi);
+    tmem_wait_ld();
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -198,16 +214,19 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
     uint32_t* cnt_p = a.counters + counter_word(g, kCntP);
     uint32_t* cnt_used = a.counters + counter_word(g, kCntUsed);
     const int n_ech = a.slice / 128;                 // E boxes (64 columns each) per CTA per O stage
-    const uint32_t o_stage_bytes = 16384u + static_cast<uint32_t>(n_ech) * 8192u;
+    const uint32_t o_stage_bytes = 16384u + static_cast<uint32_t>(n_ech) * 8192u;   // P^T 2 x 8 KB + E
     const int nG2 = 2 * G;                           // CTAs per group
 
-    if (warp == 0) {
-        // ===================================================== TMA producer (both CTAs)
+    if (warp == 0 || warp == 3) {
+        // ===================================================== TMA producers (both CTAs)
+        // Warp 0 issues the A operand of every stage (h rows, or the P^T columns of
+        // this CTA's positions) and posts the stage's expected bytes on the leader's
+        // barrier; warp 3 issues the B operand (this CTA's half of the W rows, or of
+        // the E columns).  Two issuers keep more loads in flight than one.
         if (lane == 0) {
-            tma_prefetch_desc(&a.map_h);
-            tma_prefetch_desc(&a.map_w);
-            tma_prefetch_desc(&a.map_e);
-            tma_prefetch_desc(&a.map_p);
+            const bool a_side = warp == 0;
+            tma_prefetch_desc(a_side ? &a.map_h : &a.map_w);
+            tma_prefetch_desc(a_side ? &a.map_p : &a.map_e);
             // the leader's full barrier of a stage, as a shared::cluster address
             auto full_leader = [&](int slot) { return smem_addr_in_rank(&full_bar[slot], 0); };
             uint32_t it = 0;
@@ -221,22 +240,30 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                 return true;
             };
             auto emit_o = [&](int k, int t) -> bool {
-                if (!wait_counter(cnt_p, static_cast<uint32_t>(nG2 * (k + 1)), &abort_flag, a.err, kErrProducerP))
-                    return false;
-                fence_async_global();
+                if (a_side) {
+                    if (!wait_counter(cnt_p, static_cast<uint32_t>(nG2 * (k + 1)), &abort_flag, a.err, kErrProducerP))
+                        return false;
+                    fence_async_global();
+                }
                 for (int q = 0; q < G; ++q) {
                     if (!sub_valid(t, q)) continue;
-                    const int prow = ((g * 2 + (k & 1)) * G + q) * kCanvas + static_cast<int>(prank) * kTileM;
+                    // P^T tile of (block k, sub-tile q): [256 vocab rows][256 canvas rows]
+                    const int prow = ((g * 2 + (k & 1)) * G + q) * kBV;
                     for (int c4 = 0; c4 < kBV / kVChunk; ++c4) {
                         int slot;
                         if (!acquire(slot)) return false;
                         uint8_t* st = ring + slot * kStageBytes;
-                        if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2u * o_stage_bytes);
-                        tma_load_2d_pair(st, &a.map_p, full_leader(slot), c4 * kVChunk, prow);
-                        for (int j = 0; j < n_ech; ++j)
-                            tma_load_2d_pair(st + kHalfB + j * 8192, &a.map_e, full_leader(slot),
-                                             d0 + static_cast<int>(prank) * (a.slice / 2) + j * 64,
-                                             vocab0(t, q) + c4 * kVChunk);
+                        if (a_side) {
+                            if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2u * o_stage_bytes);
+                            for (int j = 0; j < 2; ++j)
+                                tma_load_2d_pair(st + j * 8192, &a.map_p, full_leader(slot),
+                                                 static_cast<int>(prank) * kTileM + j * 64, prow + c4 * kVChunk);
+                        } else {
+                            for (int j = 0; j < n_ech; ++j)
+                                tma_load_2d_pair(st + kHalfB + j * 8192, &a.map_e, full_leader(slot),
+                                                 d0 + static_cast<int>(prank) * (a.slice / 2) + j * 64,
+                                                 vocab0(t, q) + c4 * kVChunk);
+                        }
                     }
                 }
                 return true;
@@ -253,9 +280,12 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                             int slot;
                             if (!acquire(slot)) { ok = false; break; }
                             uint8_t* st = ring + slot * kStageBytes;
-                            if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2u * kStageBytes);
-                            tma_load_2d_pair(st, &a.map_h, full_leader(slot), kc * kKChunk, row0);
-                            tma_load_2d_pair(st + kHalfB, &a.map_w, full_leader(slot), kc * kKChunk, v0);
+                            if (a_side) {
+                                if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2u * kStageBytes);
+                                tma_load_2d_pair(st, &a.map_h, full_leader(slot), kc * kKChunk, row0);
+                            } else {
+                                tma_load_2d_pair(st + kHalfB, &a.map_w, full_leader(slot), kc * kKChunk, v0);
+                            }
                         }
                     }
                     if (ok && t > tb) ok = emit_o(k - 1, t - 1);
@@ -279,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
         // ===================================================== pair UMMA issuer (leader CTA)
         if (lane == 0 && leader) {
             const uint32_t idesc_s = idesc_bf16_f32(2 * kTileM, kBV, false, false);
-            const uint32_t idesc_o = idesc_bf16_f32(2 * kTileM, a.slice, false, true);
+            const uint32_t idesc_o = idesc_bf16_f32(2 * kTileM, a.slice, true, true);
             uint32_t it = 0;
             bool ok = true;
             auto consume = [&](int& slot) -> bool {
@@ -302,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                         const uint32_t st = smem_u32(ring + slot * kStageBytes);
 #pragma unroll
                         for (int kk = 0; kk < kVChunk / 16; ++kk) {
-                            const uint64_t ad = smem_desc(st + kk * 32, 16, 1024, kSwizzle128B);
+                            const uint64_t ad = smem_desc(st + kk * 2048, 8192, 1024, kSwizzle128B);
                             const uint64_t bd = smem_desc(st + kHalfB + kk * 2048, 8192, 1024, kSwizzle128B);
                             umma_ss_pair(tmem + kTmemO, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
                         }
@@ -385,12 +415,11 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                 float smax = -INFINITY;
                 if (valid) {
 #pragma unroll 1
-                    for (int c0 = 0; c0 < kBV; c0 += 32) {
-                        uint32_t v[32];
-                        tmem_ld32(tmem + kTmemS + lane_addr + c0, v);
-                        tmem_wait_ld();
+                    for (int c0 = 0; c0 < kBV; c0 += 64) {
+                        uint32_t v[64];
+                        tmem_ld64(tmem + kTmemS + lane_addr + c0, v);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) smax = fmaxf(smax, __uint_as_float(v[i]));
+                        for (int i = 0; i < 64; ++i) smax = fmaxf(smax, __uint_as_float(v[i]));
                     }
                 }
                 float* rm = a.rowmax + static_cast<size_t>((g * 2 + (k & 1)) * G) * kCanvas;
@@ -413,38 +442,39 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                 float alpha = 1.f;
                 if (m_ref == -INFINITY || M > m_ref + kLazyRescale) {
                     if (m_ref != -INFINITY) {
-                        alpha = exp2f(m_ref - M);
+                        alpha = fast_exp2(m_ref - M);
                         u = alpha * (u + (m_ref - M) * l);
                         l = alpha * l;
                     }
                     m_ref = M;
                 }
-                // --- pass 2: probabilities, statistics, argmax, P tile
+                // --- pass 2: probabilities, statistics, argmax, P^T tile
+                // P is published transposed ([vocab][canvas row]) so that a warp's stores
+                // are contiguous: lanes 2m and 2m+1 swap one value per column pair and
+                // each stores the two rows (2m, 2m+1) of one column as a bf16 pair.
                 if (valid) {
-                    __nv_bfloat16* prow =
-                        a.pbuf + (static_cast<size_t>((g * 2 + (k & 1)) * G + r) * kCanvas + crow) * kBV;
+                    __nv_bfloat16* pt = a.pbuf + static_cast<size_t>((g * 2 + (k & 1)) * G + r) * kBV * kCanvas;
+                    const bool odd = lane & 1;
+                    const int prow = crow & ~1;
                     const int v0 = vocab0(t, r);
 #pragma unroll 1
-                    for (int c0 = 0; c0 < kBV; c0 += 32) {
-                        uint32_t v[32];
-                        tmem_ld32(tmem + kTmemS + lane_addr + c0, v);
-                        tmem_wait_ld();
-                        uint32_t pk[16];
+                    for (int c0 = 0; c0 < kBV; c0 += 64) {
+                        uint32_t v[64];
+                        tmem_ld64(tmem + kTmemS + lane_addr + c0, v);
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2) {
+                        for (int i = 0; i < 64; i += 2) {
                             const float s0 = __uint_as_float(v[i]), s1 = __uint_as_float(v[i + 1]);
                             if (s0 > best) { best = s0; best_idx = v0 + c0 + i; }
                             if (s1 > best) { best = s1; best_idx = v0 + c0 + i + 1; }
                             const float y0 = fmaf(s0, c2, -m_ref), y1 = fmaf(s1, c2, -m_ref);
-                            const float e0 = exp2f(y0), e1 = exp2f(y1);
+                            const float e0 = fast_exp2(y0), e1 = fast_exp2(y1);
                             l += e0 + e1;
                             u = fmaf(e0, y0, fmaf(e1, y1, u));
-                            pk[i / 2] = pack_bf16(e0, e1);
+                            const float recv = __shfl_xor_sync(0xffffffffu, odd ? e0 : e1, 1);
+                            const int col = c0 + i + (odd ? 1 : 0);
+                            *reinterpret_cast<uint32_t*>(pt + static_cast<size_t>(col) * kCanvas + prow) =
+                                pack_bf16(odd ? recv : e0, odd ? e1 : recv);
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(prow + c0);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                     }
                 }
                 tc_fence_before();
@@ -635,3 +665,4 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
 }
 
 }  // namespace dg
+

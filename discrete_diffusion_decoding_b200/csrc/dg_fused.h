@@ -9,9 +9,9 @@ namespace dg {
 
 struct FusedArgs {
     CUtensorMap map_h;   // h [N, d] bf16, box {64 cols, 128 rows}
-    CUtensorMap map_w;   // W [V, d] bf16, box {64 cols, 256 rows}
+    CUtensorMap map_w;   // W [V, d] bf16, box {64 cols, 128 rows} (half of a 256-row tile per CTA)
     CUtensorMap map_e;   // E [V, d] bf16, box {64 cols, 64 rows}
-    CUtensorMap map_p;   // P scratch [n_groups*2*G*128, 256] bf16, box {64 cols, 128 rows}
+    CUtensorMap map_p;   // P^T scratch [n_groups*2*G*256 vocab rows, 256 canvas rows] bf16, box {64, 64}
     const int32_t* stop;
     uint32_t* counters;
     float* rowmax;
