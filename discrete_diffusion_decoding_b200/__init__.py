@@ -15,7 +15,7 @@ from ._abi import DgError, DgParams, check, lib
 
 __all__ = ["DgError", "DgParams", "params", "workspace_size", "plan", "temperature", "dg_canvas_init",
            "dg_denoise_step", "dg_stop_check", "dg_stub_hidden", "last_launch_count", "profile_enable",
-           "profile_collect", "Workspace", "StepBuffers",
+           "profile_collect", "dg_denoise_stats_noalloc", "Workspace", "StepBuffers",
            "decode_batch", "decode_block_ar"]
 
 
@@ -107,6 +107,13 @@ def dg_stop_check(p, ws, stream=None, want_stable=False):
                                                stable if stable is not None else None, ctypes.byref(n),
                                                _stream(stream)))
     return list(flags), (list(stable) if stable is not None else None), n.value
+
+
+def dg_denoise_stats_noalloc(p, step, h, W, E, entropy, argmax, lse, selfcond, stream=None):
+    """Fused pass without a caller workspace (scratch lives in the library's fixed device array)."""
+    check("dg_denoise_stats_noalloc", lib().dg_denoise_stats_noalloc(
+        ctypes.byref(p), int(step), _ptr(h), _ptr(W), _ptr(E), _ptr(entropy), _ptr(argmax), _ptr(lse),
+        _ptr(selfcond), _stream(stream)))
 
 
 def dg_stub_hidden(p, step, gain, noise, seeds, E, tokens, h, ws, stream=None):

@@ -167,6 +167,34 @@ int dg_last_launch_count(void);
 dg_status dg_profile_enable(int max_records);
 dg_status dg_profile_collect(int* n_records, float* mean_ms, float* total_ms);
 
+/*
+ * Allocation-free variant of the fused pass of dg_denoise_step, for callers
+ * that cannot allocate device memory when they call (a plugin inside a host
+ * framework whose allocator it may not use, a process with a fixed memory
+ * budget, a latency-critical thread that must stay off the allocator).  The
+ * paper has no counterpart: this is a property of this library's interface.
+ *
+ * For every position of all n_canvas canvases (all treated as active) it
+ * computes, at step `step` (temperature T_step): entropy_dev [N] (H, nats),
+ * argmax_dev [N], lse_dev [N] (may be NULL) and selfcond_dev [N, d] fp32 (may be
+ * NULL) - the same values dg_denoise_step writes, without the sampler and stop
+ * state.  Inputs are as for dg_denoise_step.
+ *
+ * Scratch comes from a 64 MiB array the library keeps in device memory (every
+ * GPU that loads the library holds it until the process exits).  Shapes whose
+ * scratch would exceed it return DG_ENOMEM (on a 148-SM B200 with V = 262144,
+ * d = 2816, up to 4 canvases fit); the call allocates and frees nothing.  The
+ * first call on a device is its set-up: it looks up the array's device address
+ * (once per device, and the CUDA runtime may load the library's device code at
+ * that point), so make that first call before capturing a stream.  All calls on a device share the array
+ * and the call clears what must start at zero; calls whose GPU work overlaps
+ * (different streams, or no ordering between them) race on it.  An in-kernel
+ * wait that runs out is not reported by this call.
+ */
+dg_status dg_denoise_stats_noalloc(const dg_params* p, int step, const void* h_dev, const void* W_dev,
+                                   const void* E_dev, float* entropy_dev, int32_t* argmax_dev, float* lse_dev,
+                                   float* selfcond_dev, void* stream);
+
 /* Column-slice group size and group count the fused kernel uses for p on the current device. */
 dg_status dg_plan(const dg_params* p, int* group, int* n_groups, int* slice_cols);
 
