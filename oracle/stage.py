@@ -140,14 +140,15 @@ def denoise_step(h_u16, W_u16, E_u16, T, bound, seeds, s, vocab, canvas_len=256,
                  want_selfcond=True, canvas_ids=None):
     """One step over all canvases of a batch, from bf16 bit patterns.
 
-    h_u16 [N, d], W_u16 / E_u16 [V, d] (uint16 bf16 bits), seeds [C] (uint64),
+    h_u16 [N, d], W_u16 / E_u16 [V, d] (uint16 bf16 bits, or their exact float64
+    widening), seeds [C] (uint64),
     N = C * canvas_len; canvas_ids[c] (default c) is the canvas word of the
     Philox counter.  Returns dict with H, argmax, lse, top2gap, tokens,
     accept, selfcond (or None), mean_H per canvas.
     """
     h = bf16_to_f64(h_u16)
-    W = bf16_to_f64(W_u16)
-    E = W if E_u16 is W_u16 else bf16_to_f64(E_u16)
+    W = _widen(np.asarray(W_u16))
+    E = W if E_u16 is W_u16 else _widen(np.asarray(E_u16))
     n = h.shape[0]
     C = n // canvas_len
     out = {k: [] for k in ("H", "argmax", "lse", "top2gap", "tokens", "accept", "selfcond", "max")}

@@ -64,7 +64,7 @@ def canvas_seeds(n_canvas, base=0):
     return np.arange(base, base + n_canvas, dtype=np.uint64)
 
 
-def adversarial_rows(W, E_for_ties, n, seed=44):
+def adversarial_rows(W, n, seed=44):
     """Row kinds by position mod 4 for the adversarial case (recipe only).
 
     0: near-uniform - h = 0 (even i/4) or 1e-3 * N(0, 1) (odd i/4);
