@@ -16,7 +16,7 @@ using namespace dg;
 
 namespace {
 
-constexpr int kFusedSmem = 6 * 32 * 1024 + 1024 + 4 * kMaxCanvas;
+constexpr int kFusedSmem = kFusedSmemBytes;
 thread_local int g_last_launches = 0;
 
 // Event pairs recorded around fused-kernel launches while profiling is enabled.
@@ -165,6 +165,21 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, u
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D view {64 columns, rows, cols/64 column blocks} of a row-major bf16 matrix:
+// one box of {64, box_rows, box_blocks} fills box_blocks consecutive 128-byte
+// swizzle atoms (the layout the UMMA descriptors of the MN-major operands use).
+bool encode_blocks_3d(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                      uint32_t box_rows, uint32_t box_blocks) {
+    if (!enc || cols % 64 != 0) return false;
+    cuuint64_t dims[3] = {64, rows, cols / 64};
+    cuuint64_t strides[2] = {cols * 2, 128};
+    cuuint32_t box[3] = {64, box_rows, box_blocks};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <class T>
 T* at(void* ws, size_t off) {
     return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
@@ -285,8 +300,8 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
     const uint64_t prow_total = static_cast<uint64_t>(pl.n_groups) * 2 * pl.group * kCanvas;
     if (!encode_2d(&fa.map_h, h_dev, pl.N, pl.d, 64, kTileM) ||
         !encode_2d(&fa.map_w, W_dev, pl.V, pl.d, 64, kBV / 2) ||
-        !encode_2d(&fa.map_e, E_dev, pl.V, pl.d, 64, kVChunk) ||
-        !encode_2d(&fa.map_p, at<void>(workspace_dev, L.pbuf), prow_total, kCanvas, 64, kVChunk))
+        !encode_blocks_3d(encode_fn(), &fa.map_e, E_dev, pl.V, pl.d, kVChunk, pl.slice / 128) ||
+        !encode_blocks_3d(encode_fn(), &fa.map_p, at<void>(workspace_dev, L.pbuf), prow_total, kCanvas, kVChunk, 2))
         return DG_ECUDA;
     int32_t* stop = at<int32_t>(workspace_dev, L.stop);
     fa.stop = stop;
@@ -344,18 +359,20 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
     ca.n_groups = pl.n_groups;
     ca.steps_per_tile = pl.steps_per_tile;
     ca.max_seg = pl.max_seg;
-    dg_combine_kernel<<<pl.N, 256, 0, s>>>(ca);
-    if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
-
-    dg_accept_kernel<<<(pl.N + 255) / 256, 256, 0, s>>>(entropy_dev, argmax_dev, seeds_dev, stop, tokens_dev,
-                                                         accept_dev, p->eb_bound, step, pl.N, pl.V);
+    ca.seeds = seeds_dev;
+    ca.tokens = tokens_dev;
+    ca.accept = accept_dev;
+    ca.bound = p->eb_bound;
+    ca.step = step;
+    ca.V = pl.V;
+    dg_combine_kernel<<<combine_grid(pl.N, pl.d), 256, 0, s>>>(ca);
     if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
 
     dg_stop_kernel<<<pl.C, kCanvas, 0, s>>>(entropy_dev, argmax_dev, at<int32_t>(workspace_dev, L.prev_argmax),
                                             at<int32_t>(workspace_dev, L.stable), stop, p->stop_thresh, p->stability,
                                             step);
     if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
-    g_last_launches = 4;
+    g_last_launches = 3;
     return DG_OK;
 }
 

@@ -32,7 +32,7 @@
 //    the statistics written as a partial, merged by dg_combine_kernel.
 //
 // Roles inside a CTA (256 threads): warps 0 and 3 issue TMA loads (A and B
-// operands) into a 6-stage ring of 32 KB stages (both CTAs of a pair load;
+// operands) into a 7-stage ring of 32 KB stages (both CTAs of a pair load;
 // completion is counted on the leader's barriers); warp 1 allocates TMEM and,
 // in the leader CTA, issues the pair UMMAs; warps 4-7 (one TMEM lane quarter
 // each, thread = position row) do the softmax, publish P^T and run the epilogue.
@@ -49,8 +49,8 @@ namespace dg {
 
 namespace {
 
-constexpr int kStages = 6;
-constexpr int kStageBytes = 32 * 1024;     // per CTA: A operand 16 KB + B operand half 16 KB
+constexpr int kStages = kFusedStages;
+constexpr int kStageBytes = kFusedStageBytes;   // per CTA: A operand 16 KB + B operand half 16 KB
 constexpr int kHalfB = 16 * 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 0;             // logits tile columns [0, 256)
@@ -255,14 +255,13 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                         uint8_t* st = ring + slot * kStageBytes;
                         if (a_side) {
                             if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2u * o_stage_bytes);
-                            for (int j = 0; j < 2; ++j)
-                                tma_load_2d_pair(st + j * 8192, &a.map_p, full_leader(slot),
-                                                 static_cast<int>(prank) * kTileM + j * 64, prow + c4 * kVChunk);
+                            // both 64-row atoms of this CTA's canvas rows in one 3-D box
+                            tma_load_3d_pair(st, &a.map_p, full_leader(slot), 0, prow + c4 * kVChunk,
+                                             static_cast<int>(prank) * 2);
                         } else {
-                            for (int j = 0; j < n_ech; ++j)
-                                tma_load_2d_pair(st + kHalfB + j * 8192, &a.map_e, full_leader(slot),
-                                                 d0 + static_cast<int>(prank) * (a.slice / 2) + j * 64,
-                                                 vocab0(t, q) + c4 * kVChunk);
+                            // this CTA's half of the column slice (n_ech atoms of 64 columns) in one 3-D box
+                            tma_load_3d_pair(st + kHalfB, &a.map_e, full_leader(slot), 0, vocab0(t, q) + c4 * kVChunk,
+                                             (d0 + static_cast<int>(prank) * (a.slice / 2)) / 64);
                         }
                     }
                 }
@@ -548,12 +547,17 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
 }
 
 // ---------------------------------------------------------------------------
-// Split-vocabulary combine: one CTA per active position.  Merges the partial
-// statistics of every (piece, pair) covering the position's canvas:
+// Split-vocabulary combine: one CTA per (active position, block of 1024
+// self-conditioning columns).  Merges the partial statistics of every (piece,
+// pair) covering the position's canvas:
 //   M = max m_s;  L = sum_s 2^(m_s-M) sum_r l;  U = sum_s 2^(m_s-M) (sum_r u + (m_s-M) sum_r l)
 //   H = ln L - ln2 * U / L;  LSE = ln2 * (M + log2 L);  argmax = best raw logit, smallest index;
 //   sc = sum_s 2^(m_s-M) O_s / L.
-// Block 0 also clears the fused kernel's group counters for its next launch.
+// The column-block-0 CTA of a position also writes H / argmax / LSE and applies
+// the entropy-bounded sampler to it (juhoplayground, entropy bounded sampler;
+// deep dive steps 4-5): keep the argmax where H <= bound, otherwise a uniform
+// vocabulary token from Philox (tag 1, this step).  CTA (0, 0) also clears the
+// fused kernel's group counters for its next launch.
 __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
     __shared__ float sh_w[kMaxSlotsPerTile];
     __shared__ int sh_slot[kMaxSlotsPerTile];
@@ -567,7 +571,8 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
     const int c = n / kCanvas;
     const int crow = n % kCanvas;
     const int tid = threadIdx.x;
-    if (blockIdx.x == 0) {
+    const bool head = blockIdx.y == 0;      // writes the per-position scalars
+    if (blockIdx.x == 0 && head) {
         for (int i = tid; i < a.n_groups * 128; i += blockDim.x) a.counters[i] = 0u;
     }
     if (tid == 0) {
@@ -634,12 +639,22 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
             }
         }
         if (tid == 0) {
-            const float ln2 = 0.69314718055994531f;
-            const float H = logf(L) - ln2 * (Uu / L);
-            a.entropy[n] = H;
-            a.argmax[n] = bidx;
-            if (a.lse) a.lse[n] = ln2 * (M + log2f(L));
             sh_L = L;
+            if (head) {
+                const float ln2 = 0.69314718055994531f;
+                const float H = logf(L) - ln2 * (Uu / L);
+                a.entropy[n] = H;
+                a.argmax[n] = bidx;
+                if (a.lse) a.lse[n] = ln2 * (M + log2f(L));
+                if (a.tokens) {
+                    const bool acc = H <= a.bound;
+                    a.tokens[n] = acc ? bidx
+                                      : philox_token(a.seeds[c], static_cast<uint32_t>(crow),
+                                                     static_cast<uint32_t>(a.step), static_cast<uint32_t>(c),
+                                                     kTagRenoise, static_cast<uint32_t>(a.V));
+                    a.accept[n] = acc ? 1 : 0;
+                }
+            }
         }
         for (int s = tid; s < ns; s += 32)
             sh_w[s] = exp2f(a.stats[(static_cast<size_t>(sh_slot[s]) * a.G) * kCanvas + crow].x - M);
@@ -648,7 +663,8 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
     if (a.selfcond == nullptr) return;
     const int ns = n_slots_s;
     const float invL = 1.f / sh_L;
-    for (int col = tid * 4; col < a.d; col += blockDim.x * 4) {
+    const int col_end = min(a.d, static_cast<int>(blockIdx.y + 1) * kCombineCols);
+    for (int col = static_cast<int>(blockIdx.y) * kCombineCols + tid * 4; col < col_end; col += blockDim.x * 4) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int s = 0; s < ns; ++s) {
             const float4 o =

@@ -10,8 +10,9 @@ namespace dg {
 struct FusedArgs {
     CUtensorMap map_h;   // h [N, d] bf16, box {64 cols, 128 rows}
     CUtensorMap map_w;   // W [V, d] bf16, box {64 cols, 128 rows} (half of a 256-row tile per CTA)
-    CUtensorMap map_e;   // E [V, d] bf16, box {64 cols, 64 rows}
-    CUtensorMap map_p;   // P^T scratch [n_groups*2*G*256 vocab rows, 256 canvas rows] bf16, box {64, 64}
+    CUtensorMap map_e;   // E [V, d] bf16 as {64 cols, V rows, d/64 column blocks}, box {64, 64, slice/128}
+    CUtensorMap map_p;   // P^T scratch [n_groups*2*G*256 vocab rows, 256 canvas rows] bf16 as
+                         // {64 rows, vocab rows, 4 row blocks}, box {64, 64, 2}
     const int32_t* stop;
     uint32_t* counters;
     float* rowmax;
@@ -34,8 +35,18 @@ struct CombineArgs {
     int32_t* argmax;
     float* lse;
     float* selfcond;
+    // entropy-bounded accept / re-noise of each position (skipped when tokens is null)
+    const uint64_t* seeds;
+    int32_t* tokens;
+    uint8_t* accept;
+    float bound;
+    int step, V;
     int C, d, G, n_groups, steps_per_tile, max_seg;
 };
+
+// Combine grid: one CTA per (position, block of kCombineCols self-conditioning columns).
+constexpr int kCombineCols = 1024;
+inline dim3 combine_grid(int N, int d) { return dim3(N, (d + kCombineCols - 1) / kCombineCols); }
 
 __global__ void dg_fused_kernel(const __grid_constant__ FusedArgs a);
 __global__ void dg_combine_kernel(const CombineArgs a);
@@ -43,9 +54,6 @@ __global__ void dg_combine_kernel(const CombineArgs a);
 // small kernels (dg_small.cu)
 __global__ void dg_init_kernel(const uint64_t* seeds, int32_t* tokens, int32_t* prev_argmax, int32_t* stable,
                                int32_t* stop, int32_t* err, uint32_t* counters, int n_counter_words, int C, int V);
-__global__ void dg_accept_kernel(const float* entropy, const int32_t* argmax, const uint64_t* seeds,
-                                 const int32_t* stop, int32_t* tokens, uint8_t* accept, float bound, int step,
-                                 int N, int V);
 __global__ void dg_stop_kernel(const float* entropy, const int32_t* argmax, int32_t* prev_argmax, int32_t* stable,
                                int32_t* stop, float stop_thresh, int stability, int step);
 __global__ void dg_stub_kernel(const uint64_t* seeds, const __nv_bfloat16* E, const int32_t* tokens,

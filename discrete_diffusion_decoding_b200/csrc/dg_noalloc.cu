@@ -25,7 +25,7 @@
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;   // 64 MiB, stated in include/dg.h
-constexpr int kNoAllocSmem = 6 * 32 * 1024 + 1024 + 4 * dg::kMaxCanvas;
+constexpr int kNoAllocSmem = dg::kFusedSmemBytes;
 
 }  // namespace
 
@@ -72,8 +72,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-                    uint32_t box_rows) {
+EncodeTiledFn encoder() {
     static EncodeTiledFn fn = nullptr;
     static std::once_flag once;
     std::call_once(once, [] {
@@ -83,6 +82,12 @@ bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
             q == cudaDriverEntryPointSuccess)
             fn = reinterpret_cast<EncodeTiledFn>(p);
     });
+    return fn;
+}
+
+bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                    uint32_t box_rows) {
+    EncodeTiledFn fn = encoder();
     if (!fn) return false;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
@@ -91,6 +96,21 @@ bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D view {64 columns, rows, cols/64 column blocks} of a row-major bf16 matrix:
+// one box of {64, box_rows, box_blocks} fills box_blocks consecutive 128-byte
+// swizzle atoms (the layout the UMMA descriptors of the MN-major operands use).
+bool encode_blocks_3d(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                      uint32_t box_rows, uint32_t box_blocks) {
+    if (!enc || cols % 64 != 0) return false;
+    cuuint64_t dims[3] = {64, rows, cols / 64};
+    cuuint64_t strides[2] = {cols * 2, 128};
+    cuuint32_t box[3] = {64, box_rows, box_blocks};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <class T>
@@ -147,8 +167,8 @@ extern "C" dg_status dg_denoise_stats_noalloc(const dg_params* p, int step, cons
     const uint64_t prow_total = static_cast<uint64_t>(pl.n_groups) * 2 * pl.group * kCanvas;
     if (!encode_bf16_2d(&fa.map_h, h_dev, pl.N, pl.d, 64, kTileM) ||
         !encode_bf16_2d(&fa.map_w, W_dev, pl.V, pl.d, 64, kBV / 2) ||
-        !encode_bf16_2d(&fa.map_e, E_dev, pl.V, pl.d, 64, kVChunk) ||
-        !encode_bf16_2d(&fa.map_p, at<void>(ws, L.pbuf), prow_total, kCanvas, 64, kVChunk))
+        !encode_blocks_3d(encoder(), &fa.map_e, E_dev, pl.V, pl.d, kVChunk, pl.slice / 128) ||
+        !encode_blocks_3d(encoder(), &fa.map_p, at<void>(ws, L.pbuf), prow_total, kCanvas, kVChunk, 2))
         return DG_ECUDA;
     fa.stop = stop;
     fa.counters = counters;
@@ -199,7 +219,13 @@ extern "C" dg_status dg_denoise_stats_noalloc(const dg_params* p, int step, cons
     ca.n_groups = pl.n_groups;
     ca.steps_per_tile = pl.steps_per_tile;
     ca.max_seg = pl.max_seg;
-    dg_combine_kernel<<<pl.N, 256, 0, s>>>(ca);
+    ca.seeds = nullptr;
+    ca.tokens = nullptr;     // no sampler state in this entry point
+    ca.accept = nullptr;
+    ca.bound = 0.f;
+    ca.step = step;
+    ca.V = pl.V;
+    dg_combine_kernel<<<combine_grid(pl.N, pl.d), 256, 0, s>>>(ca);
     if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
     return DG_OK;
 }

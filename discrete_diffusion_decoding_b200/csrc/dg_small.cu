@@ -1,6 +1,6 @@
 // The element-wise and per-canvas kernels around the fused pass: canvas
-// initialisation, entropy-bounded accept / re-noise, the two-fold stop
-// reduction and the benchmark-only denoiser stub.
+// initialisation, the two-fold stop reduction and the benchmark-only denoiser
+// stub (the entropy-bounded accept / re-noise runs inside dg_combine_kernel).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -28,23 +28,6 @@ __global__ void dg_init_kernel(const uint64_t* seeds, int32_t* tokens, int32_t* 
     }
     if (n < 4) err[n] = 0;
     for (int w = n; w < n_counter_words; w += gridDim.x * blockDim.x) counters[w] = 0u;
-}
-
-// Entropy-bounded sampler (juhoplayground, entropy bounded sampler; deep dive
-// steps 4-5 and the 0.1 entropy bound): keep the argmax where H <= bound,
-// re-noise the rest with a uniform vocabulary token (Philox tag 1 at this step).
-__global__ void dg_accept_kernel(const float* entropy, const int32_t* argmax, const uint64_t* seeds,
-                                 const int32_t* stop, int32_t* tokens, uint8_t* accept, float bound, int step,
-                                 int N, int V) {
-    const int n = blockIdx.x * blockDim.x + threadIdx.x;
-    if (n >= N) return;
-    const int c = n / kCanvas, i = n % kCanvas;
-    if (stop[c]) return;
-    const bool acc = entropy[n] <= bound;
-    tokens[n] = acc ? argmax[n]
-                    : philox_token(seeds[c], static_cast<uint32_t>(i), static_cast<uint32_t>(step),
-                                   static_cast<uint32_t>(c), kTagRenoise, static_cast<uint32_t>(V));
-    accept[n] = acc ? 1 : 0;
 }
 
 // Two-fold adaptive stop (deep dive, "Two-Fold Adaptive Stopping"): one CTA of
