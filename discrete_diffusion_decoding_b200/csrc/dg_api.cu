@@ -152,22 +152,10 @@ dg_status make_plan(const dg_params* p, int pairs, Plan* pl) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-               uint32_t box_rows) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t es[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // 3-D view {64 columns, rows, cols/64 column blocks} of a row-major bf16 matrix:
 // one box of {64, box_rows, box_blocks} fills box_blocks consecutive 128-byte
-// swizzle atoms (the layout the UMMA descriptors of the MN-major operands use).
+// swizzle atoms (the layout the UMMA descriptors use: K-major for h and W,
+// MN-major for P^T and E).
 bool encode_blocks_3d(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                       uint32_t box_rows, uint32_t box_blocks) {
     if (!enc || cols % 64 != 0) return false;
@@ -298,8 +286,8 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
     FusedArgs fa;
     std::memset(&fa, 0, sizeof(fa));
     const uint64_t prow_total = static_cast<uint64_t>(pl.n_groups) * 2 * pl.group * kCanvas;
-    if (!encode_2d(&fa.map_h, h_dev, pl.N, pl.d, 64, kTileM) ||
-        !encode_2d(&fa.map_w, W_dev, pl.V, pl.d, 64, kBV / 2) ||
+    if (!encode_blocks_3d(encode_fn(), &fa.map_h, h_dev, pl.N, pl.d, kTileM, kKChunk / 64) ||
+        !encode_blocks_3d(encode_fn(), &fa.map_w, W_dev, pl.V, pl.d, kBV / 2, kKChunk / 64) ||
         !encode_blocks_3d(encode_fn(), &fa.map_e, E_dev, pl.V, pl.d, kVChunk, pl.slice / 128) ||
         !encode_blocks_3d(encode_fn(), &fa.map_p, at<void>(workspace_dev, L.pbuf), prow_total, kCanvas, kVChunk, 2))
         return DG_ECUDA;

@@ -13,13 +13,13 @@ namespace dg {
 constexpr int kCanvas = 256;      // positions per canvas
 constexpr int kTileM = 128;       // positions per tile (UMMA M)
 constexpr int kBV = 256;          // vocabulary rows per logits tile (UMMA N)
-constexpr int kKChunk = 64;       // hidden columns per pipeline stage of the logits GEMM
-constexpr int kVChunk = 64;       // vocabulary rows per pipeline stage of the self-conditioning GEMM
+constexpr int kKChunk = 128;      // hidden columns per pipeline stage of the logits GEMM
+constexpr int kVChunk = 128;      // vocabulary rows per pipeline stage of the self-conditioning GEMM
 constexpr int kMaxSlice = 256;    // widest self-conditioning column slice a CTA pair keeps in TMEM
 constexpr int kMaxCanvas = 256;   // canvases per call (the fused kernel keeps the active list in shared memory)
 constexpr int kThreads = 256;     // threads of the fused kernel
-constexpr int kFusedStages = 7;   // TMA ring stages of the fused kernel
-constexpr int kFusedStageBytes = 32 * 1024;
+constexpr int kFusedStages = 3;   // TMA ring stages of the fused kernel
+constexpr int kFusedStageBytes = 64 * 1024;
 constexpr int kFusedSmemBytes = kFusedStages * kFusedStageBytes + 1024 + 4 * kMaxCanvas;
 constexpr float kLazyRescale = 8.0f;  // log2 units the shared reference may lag the running max
 

@@ -32,7 +32,7 @@
 //    the statistics written as a partial, merged by dg_combine_kernel.
 //
 // Roles inside a CTA (256 threads): warps 0 and 3 issue TMA loads (A and B
-// operands) into a 7-stage ring of 32 KB stages (both CTAs of a pair load;
+// operands) into a 3-stage ring of 64 KB stages (both CTAs of a pair load;
 // completion is counted on the leader's barriers); warp 1 allocates TMEM and,
 // in the leader CTA, issues the pair UMMAs; warps 4-7 (one TMEM lane quarter
 // each, thread = position row) do the softmax, publish P^T and run the epilogue.
@@ -50,8 +50,9 @@ namespace dg {
 namespace {
 
 constexpr int kStages = kFusedStages;
-constexpr int kStageBytes = kFusedStageBytes;   // per CTA: A operand 16 KB + B operand half 16 KB
-constexpr int kHalfB = 16 * 1024;
+constexpr int kStageBytes = kFusedStageBytes;   // per CTA: A operand 32 KB + B operand half 32 KB
+constexpr int kHalfB = 32 * 1024;
+constexpr uint32_t kAtomCol = 128u * 128u;     // bytes of one 64-column swizzle atom column of a 128-row box
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 0;             // logits tile columns [0, 256)
 constexpr uint32_t kTmemO = 256;           // self-conditioning slice columns [256, 256 + slice)
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
     uint32_t* cnt_p = a.counters + counter_word(g, kCntP);
     uint32_t* cnt_used = a.counters + counter_word(g, kCntUsed);
     const int n_ech = a.slice / 128;                 // E boxes (64 columns each) per CTA per O stage
-    const uint32_t o_stage_bytes = 16384u + static_cast<uint32_t>(n_ech) * 8192u;   // P^T 2 x 8 KB + E
+    const uint32_t o_stage_bytes = 2u * kAtomCol + static_cast<uint32_t>(n_ech) * kAtomCol;   // P^T 2 x 16 KB + E
     const int nG2 = 2 * G;                           // CTAs per group
 
     if (warp == 0 || warp == 3) {
@@ -249,18 +250,18 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                     if (!sub_valid(t, q)) continue;
                     // P^T tile of (block k, sub-tile q): [256 vocab rows][256 canvas rows]
                     const int prow = ((g * 2 + (k & 1)) * G + q) * kBV;
-                    for (int c4 = 0; c4 < kBV / kVChunk; ++c4) {
+                    for (int vc = 0; vc < kBV / kVChunk; ++vc) {
                         int slot;
                         if (!acquire(slot)) return false;
                         uint8_t* st = ring + slot * kStageBytes;
                         if (a_side) {
                             if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2u * o_stage_bytes);
                             // both 64-row atoms of this CTA's canvas rows in one 3-D box
-                            tma_load_3d_pair(st, &a.map_p, full_leader(slot), 0, prow + c4 * kVChunk,
+                            tma_load_3d_pair(st, &a.map_p, full_leader(slot), 0, prow + vc * kVChunk,
                                              static_cast<int>(prank) * 2);
                         } else {
                             // this CTA's half of the column slice (n_ech atoms of 64 columns) in one 3-D box
-                            tma_load_3d_pair(st + kHalfB, &a.map_e, full_leader(slot), 0, vocab0(t, q) + c4 * kVChunk,
+                            tma_load_3d_pair(st + kHalfB, &a.map_e, full_leader(slot), 0, vocab0(t, q) + vc * kVChunk,
                                              (d0 + static_cast<int>(prank) * (a.slice / 2)) / 64);
                         }
                     }
@@ -281,9 +282,9 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                             uint8_t* st = ring + slot * kStageBytes;
                             if (a_side) {
                                 if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2u * kStageBytes);
-                                tma_load_2d_pair(st, &a.map_h, full_leader(slot), kc * kKChunk, row0);
+                                tma_load_3d_pair(st, &a.map_h, full_leader(slot), 0, row0, kc * (kKChunk / 64));
                             } else {
-                                tma_load_2d_pair(st + kHalfB, &a.map_w, full_leader(slot), kc * kKChunk, v0);
+                                tma_load_3d_pair(st + kHalfB, &a.map_w, full_leader(slot), 0, v0, kc * (kKChunk / 64));
                             }
                         }
                     }
@@ -325,14 +326,14 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                 bool first = seg_first;
                 for (int q = 0; q < G; ++q) {
                     if (!sub_valid(t, q)) continue;
-                    for (int c4 = 0; c4 < kBV / kVChunk; ++c4) {
+                    for (int vc = 0; vc < kBV / kVChunk; ++vc) {
                         int slot;
                         if (!consume(slot)) return false;
                         const uint32_t st = smem_u32(ring + slot * kStageBytes);
 #pragma unroll
                         for (int kk = 0; kk < kVChunk / 16; ++kk) {
-                            const uint64_t ad = smem_desc(st + kk * 2048, 8192, 1024, kSwizzle128B);
-                            const uint64_t bd = smem_desc(st + kHalfB + kk * 2048, 8192, 1024, kSwizzle128B);
+                            const uint64_t ad = smem_desc(st + kk * 2048, kAtomCol, 1024, kSwizzle128B);
+                            const uint64_t bd = smem_desc(st + kHalfB + kk * 2048, kAtomCol, 1024, kSwizzle128B);
                             umma_ss_pair(tmem + kTmemO, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
                         }
                         first = false;
@@ -361,8 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                             const uint32_t st = smem_u32(ring + slot * kStageBytes);
 #pragma unroll
                             for (int kk = 0; kk < kKChunk / 16; ++kk) {
-                                const uint64_t ad = smem_desc(st + kk * 32, 16, 1024, kSwizzle128B);
-                                const uint64_t bd = smem_desc(st + kHalfB + kk * 32, 16, 1024, kSwizzle128B);
+                                // K step kk: atom column kk / 4, 32-byte offset (kk % 4) inside the swizzled row
+                                const uint32_t ko = (kk >> 2) * kAtomCol + (kk & 3) * 32;
+                                const uint64_t ad = smem_desc(st + ko, 16, 1024, kSwizzle128B);
+                                const uint64_t bd = smem_desc(st + kHalfB + ko, 16, 1024, kSwizzle128B);
                                 umma_ss_pair(tmem + kTmemS, ad, bd, idesc_s, (kc | kk) != 0 ? 1u : 0u);
                             }
                             umma_commit_pair(&empty_bar[slot], 0x3);

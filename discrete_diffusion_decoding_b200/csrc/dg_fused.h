@@ -8,11 +8,13 @@
 namespace dg {
 
 struct FusedArgs {
-    CUtensorMap map_h;   // h [N, d] bf16, box {64 cols, 128 rows}
-    CUtensorMap map_w;   // W [V, d] bf16, box {64 cols, 128 rows} (half of a 256-row tile per CTA)
-    CUtensorMap map_e;   // E [V, d] bf16 as {64 cols, V rows, d/64 column blocks}, box {64, 64, slice/128}
-    CUtensorMap map_p;   // P^T scratch [n_groups*2*G*256 vocab rows, 256 canvas rows] bf16 as
-                         // {64 rows, vocab rows, 4 row blocks}, box {64, 64, 2}
+    // every operand as a 3-D view {64 columns, rows, column blocks of 64} of a
+    // row-major bf16 matrix, so that one box fills several 128-byte swizzle atoms
+    CUtensorMap map_h;   // h [N, d], box {64, 128 rows, 2}: a 128 x 128 K-major tile
+    CUtensorMap map_w;   // W [V, d], box {64, 128 rows, 2} (half of a 256-row tile per CTA)
+    CUtensorMap map_e;   // E [V, d], box {64, 128 vocab rows, slice/128}: MN-major B operand
+    CUtensorMap map_p;   // P^T scratch [n_groups*2*G*256 vocab rows, 256 canvas rows],
+                         // box {64, 128 vocab rows, 2}: MN-major A operand
     const int32_t* stop;
     uint32_t* counters;
     float* rowmax;
