@@ -20,6 +20,9 @@ constexpr int kMaxCanvas = 256;   // canvases per call (the fused kernel keeps t
 constexpr int kThreads = 256;     // threads of the fused kernel
 constexpr int kFusedStages = 3;   // TMA ring stages of the fused kernel
 constexpr int kFusedStageBytes = 64 * 1024;
+// With E aliasing W, this many tenths of the hidden columns of every W tile keep normal
+// L2 priority between the logits and the self-conditioning pass (the rest is streamed).
+constexpr int kKeepWTenths = 3;
 constexpr int kFusedSmemBytes = kFusedStages * kFusedStageBytes + 1024 + 4 * kMaxCanvas;
 constexpr float kLazyRescale = 8.0f;  // log2 units the shared reference may lag the running max
 

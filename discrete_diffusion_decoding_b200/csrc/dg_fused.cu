@@ -228,6 +228,11 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
             const bool a_side = warp == 0;
             tma_prefetch_desc(a_side ? &a.map_h : &a.map_w);
             tma_prefetch_desc(a_side ? &a.map_p : &a.map_e);
+            // L2 policy: E rows are dead once the self-conditioning pass has read them, and so
+            // are W rows unless E aliases W; with aliasing, the first keep_w_stages column
+            // stages of every W tile keep normal priority (the two blocks in flight of every
+            // group would not fit in L2 whole) and are read again from L2 as E
+            const uint64_t pol_stream = l2_policy_evict_first();
             // the leader's full barrier of a stage, as a shared::cluster address
             auto full_leader = [&](int slot) { return smem_addr_in_rank(&full_bar[slot], 0); };
             uint32_t it = 0;
@@ -261,8 +266,9 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                                              static_cast<int>(prank) * 2);
                         } else {
                             // this CTA's half of the column slice (n_ech atoms of 64 columns) in one 3-D box
-                            tma_load_3d_pair(st + kHalfB, &a.map_e, full_leader(slot), 0, vocab0(t, q) + vc * kVChunk,
-                                             (d0 + static_cast<int>(prank) * (a.slice / 2)) / 64);
+                            tma_load_3d_pair_hint(st + kHalfB, &a.map_e, full_leader(slot), 0,
+                                                  vocab0(t, q) + vc * kVChunk,
+                                                  (d0 + static_cast<int>(prank) * (a.slice / 2)) / 64, pol_stream);
                         }
                     }
                 }
@@ -284,7 +290,12 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                                 if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2u * kStageBytes);
                                 tma_load_3d_pair(st, &a.map_h, full_leader(slot), 0, row0, kc * (kKChunk / 64));
                             } else {
-                                tma_load_3d_pair(st + kHalfB, &a.map_w, full_leader(slot), 0, v0, kc * (kKChunk / 64));
+                                if (kc < a.keep_w_stages)
+                                    tma_load_3d_pair(st + kHalfB, &a.map_w, full_leader(slot), 0, v0,
+                                                     kc * (kKChunk / 64));
+                                else
+                                    tma_load_3d_pair_hint(st + kHalfB, &a.map_w, full_leader(slot), 0, v0,
+                                                          kc * (kKChunk / 64), pol_stream);
                             }
                         }
                     }

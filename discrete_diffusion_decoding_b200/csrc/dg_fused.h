@@ -24,6 +24,9 @@ struct FusedArgs {
     float* opart;
     int* err;
     int C, V, d, G, slice, n_groups, steps_per_tile, max_seg;
+    int keep_w_stages;   // E aliases W: the first keep_w_stages hidden-column stages of every W
+                         // tile keep normal L2 priority, so the self-conditioning pass finds them
+                         // there (0 when E is a separate matrix)
     float scale_log2;    // log2(e) / T
 };
 

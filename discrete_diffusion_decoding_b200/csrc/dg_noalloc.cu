@@ -170,6 +170,7 @@ extern "C" dg_status dg_denoise_stats_noalloc(const dg_params* p, int step, cons
     fa.V = pl.V;
     fa.d = pl.d;
     fa.G = pl.group;
+    fa.keep_w_stages = E_dev == W_dev ? (pl.d / kKChunk) * kKeepWTenths / 10 : 0;
     fa.slice = pl.slice;
     fa.n_groups = pl.n_groups;
     fa.steps_per_tile = pl.steps_per_tile;
