@@ -36,7 +36,18 @@ FLOPS_PER_STEP = 2 * (2.0 * N_POS * V * D)          # two contractions: logits a
 WE_BYTES_PER_STEP = 2.0 * V * D                     # tied bf16 W = E streamed once
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "dg_fused_kernel_single_step_v262144_d2816.md")
-FUSED_SRC = os.path.join(ROOT, "discrete_diffusion_decoding_b200", "csrc", "dg_fused.cu")
+CSRC = os.path.join(ROOT, "discrete_diffusion_decoding_b200", "csrc")
+
+
+def kernel_source_hash():
+    """sha256 over every CUDA source and header of the library, in name order."""
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
 
 
 def _set_vocab(vocab):
@@ -87,7 +98,7 @@ def profiled_traffic():
     """DRAM bytes per fused launch from the committed ncu summary, if it was taken on this kernel source."""
     try:
         text = open(PROFILE_SUMMARY).read()
-        src_hash = hashlib.sha256(open(FUSED_SRC, "rb").read()).hexdigest()
+        src_hash = kernel_source_hash()
     except OSError:
         return None
     fields = {}
