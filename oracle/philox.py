@@ -16,6 +16,9 @@ Keying (a reading, the pages are silent): key = (lo32(seed), hi32(seed)) of the
 per-canvas seed; counter = (position i, step s, canvas c, tag).  Tags separate
 the streams: 0 canvas init, 1 re-noise, 2 stub target ids, 3 stub Gaussian noise.
 A token is word 0 mapped to [0, V) by the multiply-high floor(r * V / 2^32).
+The sampled-acceptance mode draws one word per (position, vocabulary entry):
+word (v mod 4) of counter (floor(v / 4), s, c, 4 + 256 i) - the fourth counter
+word is >= 4 there, so these streams never meet the four above.
 
 Pins: known-answer vectors of the SC'11 reference implementation
 (tests/golden/philox4x32_10_kat.txt), bijectivity on a reduced counter set,
@@ -34,6 +37,7 @@ TAG_INIT = 0
 TAG_RENOISE = 1
 TAG_STUB_TARGET = 2
 TAG_STUB_NOISE = 3
+TAG_SAMPLE = 4
 
 
 def _round(c0, c1, c2, c3, k0, k1):
@@ -83,3 +87,11 @@ def uniform_token(seed, i, s, c, tag, vocab):
     """floor(word0 * V / 2^32): a token uniform on [0, V) (exact when V is a power of 2)."""
     w0 = words(seed, i, s, c, tag)[..., 0].astype(np.uint64)
     return ((w0 * np.uint64(vocab)) >> np.uint64(32)).astype(np.int64)
+
+
+def vocab_words(seed, i, s, c, vocab):
+    """One 32-bit word per vocabulary entry v of position i: word (v mod 4) of counter
+    (floor(v / 4), s, c, TAG_SAMPLE + 256 i).  Returns uint32 [vocab] (vocab a multiple of 4)."""
+    q = np.arange(vocab // 4, dtype=np.uint64)
+    w = words(seed, q, s, c, TAG_SAMPLE + 256 * int(i))          # [vocab/4, 4]
+    return w.reshape(-1)

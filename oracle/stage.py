@@ -18,8 +18,16 @@ Everything is float64 on the exact bf16 inputs the GPU receives (bf16 bit
 patterns widened to double).  The N x V logits block is formed explicitly: that
 is allowed here, and only here.
 
+The sampled-acceptance mode (``gumbel_noise``, ``gumbel_sample``; the accepted
+token is a draw from softmax(z / T) rather than the argmax) is a reading of the
+same passages - [DD] step 4 keeps "high-confidence" tokens and [JP] names
+temperature sharpening - that the pages leave open; the argmax mode stays the
+default.
+
 Parity status: every function below is pinned by tests/test_oracle_stage.py
-(closed forms, brute force, invariants) except ``stub_hidden``'s realism as a
+(closed forms, brute force, invariants) and, for the sampler, by
+tests/test_oracle_sample.py (Gumbel moments and CDF, chi-square of the draws
+against softmax, planted mistakes, limits), except ``stub_hidden``'s realism as a
 stand-in for a trained denoiser, which is "parity unpinned" by nature: the
 pages print no sampler trajectory.
 """
@@ -111,6 +119,43 @@ def init_tokens(seed, c, vocab, n=256):
     return philox.uniform_token(seed, np.arange(n), 0, c, philox.TAG_INIT, vocab)
 
 
+def gumbel_noise(seed, i, s, c, vocab):
+    """Standard Gumbel noise g_v = -ln(-ln u_v) for every vocabulary entry of position i.
+
+    u_v = (w_v + 1/2) / 2^32 with w_v from philox.vocab_words: uniform on (0, 1),
+    never 0 or 1.  -ln u_v is evaluated as -log1p(-(1 - u_v)), where
+    1 - u_v = (2^32 - 1 - w_v + 1/2) / 2^32 is exact in double, so the noise keeps
+    full relative precision as u_v -> 1 (where the winners of a large vocabulary lie).
+    """
+    w = philox.vocab_words(seed, i, s, c, vocab).astype(np.float64)
+    one_minus_u = (4294967295.0 - w + 0.5) / 4294967296.0
+    return -np.log(-np.log1p(-one_minus_u))
+
+
+def gumbel_sample(z, seed, s, c, positions):
+    """Sampled acceptance: a draw from softmax(z_i) for each row by the Gumbel-max trick.
+
+    The accepted token is argmax_v (z[i, v] + g[i, v]) (smallest v on an exact tie),
+    with g the per-(position, entry) Gumbel noise of gumbel_noise and z the
+    temperature-scaled logits (the distribution whose entropy the bound tests).
+    argmax of z + Gumbel noise is distributed as softmax(z) (Gumbel 1954; the
+    "Gumbel-max trick" of Maddison, Tarlow and Minka 2014).  Returns (sample int64 [n],
+    keygap float64 [n]: best key minus the second best, for the near-tie exclusion).
+    """
+    z = np.asarray(z, np.float64)
+    n, V = z.shape
+    out = np.empty(n, np.int64)
+    gap = np.empty(n)
+    for r, i in enumerate(positions):
+        key = z[r] + gumbel_noise(seed, int(i), s, c, V)
+        b = int(np.argmax(key))
+        out[r] = b
+        k2 = key.copy()
+        k2[b] = -np.inf
+        gap[r] = key[b] - k2.max() if V > 1 else np.inf
+    return out, gap
+
+
 def eb_accept(H, argmax, bound, renoise):
     """Entropy-bounded accept / re-noise ([JP] sampler; [DD] steps 4-5, bound 0.1).
 
@@ -200,19 +245,30 @@ def self_conditioning_chunked(p, E, chunk=16384):
     return sc
 
 
-def step_rows(h_u16, W_u16, E_u16, T, bound, seed, s, c, positions, vocab, want_selfcond=True):
+def step_rows(h_u16, W_u16, E_u16, T, bound, seed, s, c, positions, vocab, want_selfcond=True,
+              accept_mode=0):
     """One step for selected positions of one canvas (rows of h_u16 are those positions).
 
     W_u16 / E_u16 may be bf16 bit patterns or their exact float64 widening.
 
-    positions: index of each row within its canvas (for the re-noise draw).
-    Returns dict with H, argmax, lse, top2gap, tokens, accept, selfcond.
+    positions: index of each row within its canvas (for the re-noise and sample draws).
+    accept_mode 0 keeps the argmax at accepted positions, 1 a Gumbel-max sample of
+    softmax(z / T) (gumbel_sample).
+    Returns dict with H, argmax, lse, top2gap, tokens, accept, selfcond, and with
+    accept_mode 1 also sample and keygap.
     """
     h = bf16_to_f64(h_u16)
-    st = distribution_stats(logits_chunked(h, W_u16, T))
+    z = logits_chunked(h, W_u16, T)
+    out = {}
+    kept = None
+    if accept_mode == 1:
+        out["sample"], out["keygap"] = gumbel_sample(z, seed, s, c, positions)
+        kept = out["sample"]
+    st = distribution_stats(z)
+    del z
     ren = philox.uniform_token(seed, np.asarray(positions), s, c, philox.TAG_RENOISE, vocab)
-    tok, acc = eb_accept(st["H"], st["argmax"], bound, ren)
-    out = {k: st[k] for k in ("H", "argmax", "lse", "top2gap", "max")}
+    tok, acc = eb_accept(st["H"], st["argmax"] if kept is None else kept, bound, ren)
+    out.update({k: st[k] for k in ("H", "argmax", "lse", "top2gap", "max")})
     out["tokens"], out["accept"] = tok, acc
     out["selfcond"] = self_conditioning_chunked(st["p"], E_u16) if want_selfcond else None
     return out
