@@ -67,6 +67,9 @@ bool fused_attr_set() {
     static cudaError_t err = cudaSuccess;
     std::call_once(once, [] {
         err = cudaFuncSetAttribute(dg_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem);
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(dg_fused_sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kFusedSmem);
     });
     return err == cudaSuccess;
 }
@@ -108,6 +111,7 @@ bool params_ok(const dg_params* p) {
     if (p->max_steps < 1) return false;
     if (!(p->t_start > 0.f) || !(p->t_end > 0.f)) return false;
     if (p->stability < 0) return false;
+    if (p->accept_mode != 0 && p->accept_mode != 1) return false;
     return true;
 }
 
@@ -192,6 +196,7 @@ void dg_params_default(dg_params* p, int n_canvas, int vocab, int hidden) {
     p->stability = 2;
     p->tied = 1;
     p->group = 0;
+    p->accept_mode = 0;
 }
 
 float dg_temperature(const dg_params* p, int step) {
@@ -300,6 +305,10 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
     fa.stat_idx = at<int32_t>(workspace_dev, L.stat_idx);
     fa.opart = at<float>(workspace_dev, L.opart);
     fa.err = at<int>(workspace_dev, L.err);
+    fa.seeds = seeds_dev;
+    fa.skey = at<float>(workspace_dev, L.skey);
+    fa.sidx = at<int32_t>(workspace_dev, L.sidx);
+    fa.step = step;
     fa.C = pl.C;
     fa.V = pl.V;
     fa.d = pl.d;
@@ -326,7 +335,8 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
     cfg.numAttrs = 1;
     const bool prof = g_prof.on && g_prof.used < g_prof.max_records;
     if (prof && cudaEventRecord(g_prof.start[g_prof.used], s) != cudaSuccess) return DG_ECUDA;
-    if (cudaLaunchKernelEx(&cfg, dg_fused_kernel, fa) != cudaSuccess) return DG_ECUDA;
+    if (cudaLaunchKernelEx(&cfg, p->accept_mode == 1 ? dg_fused_sample_kernel : dg_fused_kernel, fa) != cudaSuccess)
+        return DG_ECUDA;
     if (prof) {
         if (cudaEventRecord(g_prof.stop[g_prof.used], s) != cudaSuccess) return DG_ECUDA;
         ++g_prof.used;
@@ -337,6 +347,9 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
     ca.counters = fa.counters;
     ca.stats = fa.stats;
     ca.stat_idx = fa.stat_idx;
+    ca.skey = fa.skey;
+    ca.sidx = fa.sidx;
+    ca.accept_mode = p->accept_mode;
     ca.opart = fa.opart;
     ca.entropy = entropy_dev;
     ca.argmax = argmax_dev;

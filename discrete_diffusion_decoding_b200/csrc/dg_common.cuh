@@ -59,6 +59,8 @@ __host__ __device__ inline int32_t philox_token(uint64_t seed, uint32_t i, uint3
 }
 
 enum : uint32_t { kTagInit = 0, kTagRenoise = 1, kTagStubTarget = 2, kTagStubNoise = 3 };
+// sampled acceptance: counter (v / 4, step, canvas, kTagSample + 256 i), one word per entry v
+constexpr uint32_t kTagSample = 4;
 
 // ------------------------------------------------------------------ plan and layout
 struct Plan {
@@ -78,6 +80,8 @@ struct Layout {
     size_t pbuf;                                  // [n_groups][2][G][kBV vocab][256 rows] bf16 (P^T)
     size_t stats;                                 // [n_slots][G][256] float4 {m, l, u, best}
     size_t stat_idx;                              // [n_slots][G][256] int32
+    size_t skey;                                  // [n_slots][G][256] float: best Gumbel-max key (sampled mode)
+    size_t sidx;                                  // [n_slots][G][256] int32: its vocabulary index
     size_t opart;                                 // [n_slots][256][d] float
     size_t total;
 };
@@ -101,6 +105,8 @@ inline Layout make_layout(const Plan& pl) {
     L.pbuf = take(static_cast<size_t>(2) * pl.n_groups * 2 * pl.group * kCanvas * kBV);
     L.stats = take(sizeof(float) * 4 * static_cast<size_t>(pl.n_slots) * pl.group * kCanvas);
     L.stat_idx = take(sizeof(int32_t) * static_cast<size_t>(pl.n_slots) * pl.group * kCanvas);
+    L.skey = take(sizeof(float) * static_cast<size_t>(pl.n_slots) * pl.group * kCanvas);
+    L.sidx = take(sizeof(int32_t) * static_cast<size_t>(pl.n_slots) * pl.group * kCanvas);
     L.opart = take(sizeof(float) * static_cast<size_t>(pl.n_slots) * kCanvas * pl.d);
     L.total = o;
     return L;

@@ -105,6 +105,13 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
+// log2(x) on the SFU (documented PTX lg2.approx; relative error about 2^-22).
+__device__ __forceinline__ float fast_log2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // 64 consecutive TMEM columns of this thread's lane, two loads in flight per wait.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&v)[64]) {
     uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
@@ -148,7 +155,21 @@ struct Schedule {
 
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_constant__ FusedArgs a) {
+// Gumbel-max key of one logit, in log2 units up to a constant: s log2(e)/T - log2(-log2 u)
+// with u = 1 - eps, eps = (~w + 1/2) 2^-32 (u = (w + 1/2) 2^-32 exactly), so that
+// argmax_v key = argmax_v (z_v + g_v) with g = -ln(-ln u) standard Gumbel noise.
+// -log2(1 - eps) comes from the SFU logarithm, or below eps = 2^-8 from its series
+// log2(e) (eps + eps^2/2 + eps^3/3) (relative truncation error < 2^-26), which keeps
+// full precision where u -> 1, the region the winners of a large vocabulary come from.
+__device__ __forceinline__ float gumbel_key(float s, float c2, uint32_t w) {
+    const float eps = fmaf(static_cast<float>(~w), 2.3283064365386963e-10f, 1.1641532182693481e-10f);
+    const float series = eps * fmaf(eps, fmaf(eps, 0.333333343f, 0.5f), 1.0f) * 1.44269502f;
+    const float e2 = eps < 0.00390625f ? series : -fast_log2(1.0f - eps);
+    return fmaf(s, c2, -fast_log2(e2));
+}
+
+template <bool kSample>
+__device__ __forceinline__ void fused_pass(const FusedArgs& a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     int* active = reinterpret_cast<int*>(ring + kStages * kStageBytes);
@@ -418,6 +439,17 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
             if (!sch.seg(j, ct, tb, te)) continue;
             float m_ref = -INFINITY, l = 0.f, u = 0.f, best = -INFINITY;
             int best_idx = -1;
+            // sampled acceptance: Philox key of this canvas, counter word 3 of this position
+            float skey = -INFINITY;
+            int sidx = -1;
+            uint32_t key_lo = 0, key_hi = 0, pos_word = 0, canvas = 0;
+            if constexpr (kSample) {
+                canvas = static_cast<uint32_t>(active[ct]);
+                const uint64_t seed = a.seeds[canvas];
+                key_lo = static_cast<uint32_t>(seed);
+                key_hi = static_cast<uint32_t>(seed >> 32);
+                pos_word = kTagSample + 256u * static_cast<uint32_t>(crow);
+            }
             for (int t = tb; t < te; ++t, ++k) {
                 const bool valid = sub_valid(t, r);
                 mbar_wait(&s_full, k & 1, &abort_flag, a.err, kErrSmaxSFull);
@@ -488,6 +520,21 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
                             *reinterpret_cast<uint32_t*>(pt + static_cast<size_t>(col) * kCanvas + prow) =
                                 pack_bf16(odd ? recv : e0, odd ? e1 : recv);
                         }
+                        if constexpr (kSample) {
+                            // Gumbel-max over the same logits: word (v mod 4) of Philox counter
+                            // (v / 4, step, canvas, 4 + 256 i); strict > keeps the smallest v on a tie
+#pragma unroll
+                            for (int i = 0; i < 64; i += 4) {
+                                const uint32_t v4 = static_cast<uint32_t>(v0 + c0 + i);
+                                uint32_t w[4] = {v4 >> 2, static_cast<uint32_t>(a.step), canvas, pos_word};
+                                philox4x32_10(w, key_lo, key_hi);
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    const float kj = gumbel_key(__uint_as_float(v[i + j]), c2, w[j]);
+                                    if (kj > skey) { skey = kj; sidx = static_cast<int>(v4) + j; }
+                                }
+                            }
+                        }
                     }
                 }
                 tc_fence_before();
@@ -548,6 +595,10 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
             const size_t si = (static_cast<size_t>(slot) * G + r) * kCanvas + crow;
             a.stats[si] = make_float4(m_ref, l, u, best);
             a.stat_idx[si] = best_idx;
+            if constexpr (kSample) {
+                a.skey[si] = skey;
+                a.sidx[si] = sidx;
+            }
             tc_fence_before();
             softmax_bar();
         }
@@ -560,6 +611,14 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
     if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
 }
 
+__global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_constant__ FusedArgs a) {
+    fused_pass<false>(a);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) dg_fused_sample_kernel(const __grid_constant__ FusedArgs a) {
+    fused_pass<true>(a);
+}
+
 // ---------------------------------------------------------------------------
 // Split-vocabulary combine: one CTA per (active position, block of 1024
 // self-conditioning columns).  Merges the partial statistics of every (piece,
@@ -569,9 +628,10 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_cons
 //   sc = sum_s 2^(m_s-M) O_s / L.
 // The column-block-0 CTA of a position also writes H / argmax / LSE and applies
 // the entropy-bounded sampler to it (juhoplayground, entropy bounded sampler;
-// deep dive steps 4-5): keep the argmax where H <= bound, otherwise a uniform
-// vocabulary token from Philox (tag 1, this step).  CTA (0, 0) also clears the
-// fused kernel's group counters for its next launch.
+// deep dive steps 4-5): keep the argmax where H <= bound (in the sampled mode the
+// Gumbel-max sample: the largest key over all pieces, smallest index on a tie),
+// otherwise a uniform vocabulary token from Philox (tag 1, this step).  CTA (0, 0)
+// also clears the fused kernel's group counters for its next launch.
 __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
     __shared__ float sh_w[kMaxSlotsPerTile];
     __shared__ int sh_slot[kMaxSlotsPerTile];
@@ -626,8 +686,8 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
         ns = n_slots_s;
         for (int s = 0; s < ns; ++s)
             M = fmaxf(M, a.stats[(static_cast<size_t>(sh_slot[s]) * a.G) * kCanvas + crow].x);
-        float L = 0.f, Uu = 0.f, best = -INFINITY;
-        int bidx = 0x7fffffff;
+        float L = 0.f, Uu = 0.f, best = -INFINITY, skey = -INFINITY;
+        int bidx = 0x7fffffff, sidx = 0x7fffffff;
         for (int e = tid; e < ns * a.G; e += 32) {
             const int s = e / a.G, rr = e % a.G;
             const size_t si = (static_cast<size_t>(sh_slot[s]) * a.G + rr) * kCanvas + crow;
@@ -640,6 +700,14 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
                 best = st.w;
                 bidx = idx;
             }
+            if (a.accept_mode == 1) {
+                const float kk = a.skey[si];
+                const int ki = a.sidx[si];
+                if (ki >= 0 && (kk > skey || (kk == skey && ki < sidx))) {
+                    skey = kk;
+                    sidx = ki;
+                }
+            }
         }
 #pragma unroll
         for (int off = 16; off; off >>= 1) {
@@ -650,6 +718,12 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
             if (ob > best || (ob == best && oi < bidx)) {
                 best = ob;
                 bidx = oi;
+            }
+            const float ok = __shfl_xor_sync(0xffffffffu, skey, off);
+            const int oki = __shfl_xor_sync(0xffffffffu, sidx, off);
+            if (ok > skey || (ok == skey && oki < sidx)) {
+                skey = ok;
+                sidx = oki;
             }
         }
         if (tid == 0) {
@@ -662,7 +736,7 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
                 if (a.lse) a.lse[n] = ln2 * (M + log2f(L));
                 if (a.tokens) {
                     const bool acc = H <= a.bound;
-                    a.tokens[n] = acc ? bidx
+                    a.tokens[n] = acc ? (a.accept_mode == 1 ? sidx : bidx)
                                       : philox_token(a.seeds[c], static_cast<uint32_t>(crow),
                                                      static_cast<uint32_t>(a.step), static_cast<uint32_t>(c),
                                                      kTagRenoise, static_cast<uint32_t>(a.V));

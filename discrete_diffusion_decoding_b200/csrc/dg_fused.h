@@ -23,6 +23,12 @@ struct FusedArgs {
     int32_t* stat_idx;
     float* opart;
     int* err;
+    // sampled acceptance (dg_fused_sample_kernel only): per-canvas Philox seeds, the
+    // step, and the best Gumbel-max key / index of every (piece, pair, position)
+    const uint64_t* seeds;
+    float* skey;
+    int32_t* sidx;
+    int step;
     int C, V, d, G, slice, n_groups, steps_per_tile, max_seg;
     int keep_w_stages;   // E aliases W: the first keep_w_stages hidden-column stages of every W
                          // tile keep normal L2 priority, so the self-conditioning pass finds them
@@ -35,6 +41,9 @@ struct CombineArgs {
     uint32_t* counters;
     const float4* stats;
     const int32_t* stat_idx;
+    const float* skey;       // sampled acceptance: Gumbel-max keys / indices (accept_mode 1)
+    const int32_t* sidx;
+    int accept_mode;         // 0: keep the argmax, 1: keep the Gumbel-max sample
     const float* opart;
     float* entropy;
     int32_t* argmax;
@@ -53,7 +62,8 @@ struct CombineArgs {
 constexpr int kCombineCols = 1024;
 inline dim3 combine_grid(int N, int d) { return dim3(N, (d + kCombineCols - 1) / kCombineCols); }
 
-__global__ void dg_fused_kernel(const __grid_constant__ FusedArgs a);
+__global__ void dg_fused_kernel(const __grid_constant__ FusedArgs a);          // argmax acceptance
+__global__ void dg_fused_sample_kernel(const __grid_constant__ FusedArgs a);   // + Gumbel-max sample
 __global__ void dg_combine_kernel(const CombineArgs a);
 
 // small kernels (dg_small.cu)

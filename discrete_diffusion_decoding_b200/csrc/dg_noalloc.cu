@@ -197,6 +197,9 @@ extern "C" dg_status dg_denoise_stats_noalloc(const dg_params* p, int step, cons
     ca.counters = counters;
     ca.stats = fa.stats;
     ca.stat_idx = fa.stat_idx;
+    ca.skey = nullptr;          // statistics only: no acceptance, so no sample
+    ca.sidx = nullptr;
+    ca.accept_mode = 0;
     ca.opart = fa.opart;
     ca.entropy = entropy_dev;
     ca.argmax = argmax_dev;

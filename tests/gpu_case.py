@@ -4,7 +4,9 @@ run the oracle on the same inputs, and compare under the stated tolerances.
 Tolerances (per position): H within 1e-3 nats; self-conditioning within 2e-2
 relative L2; tokens, accept flags and argmax bit-exact except at positions whose
 oracle entropy is within 1e-3 of the bound or whose top-2 logits (z = h.W/T)
-differ by less than 1e-3 - those are listed and excluded.
+differ by less than 1e-3 - those are listed and excluded.  In the sampled
+acceptance mode the kept token is the Gumbel-max sample; positions whose two
+best keys (z + g) differ by less than 1e-3 are excluded the same way.
 """
 
 import numpy as np
@@ -42,17 +44,20 @@ def gpu_step(dg, p, step, h, Wd, Ed, seeds, tokens_in=None, ws=None, bufs=None):
     return out
 
 
-def oracle_rows(h_bits, W_bits, E_bits, T, bound, seeds, step, rows, vocab, canvas_len=256, want_selfcond=True):
+def oracle_rows(h_bits, W_bits, E_bits, T, bound, seeds, step, rows, vocab, canvas_len=256, want_selfcond=True,
+                accept_mode=0):
     """Oracle for selected global rows (positions); canvas index and seed derive from the row."""
     rows = np.asarray(rows)
     n, d = len(rows), h_bits.shape[1]
     out = {"H": np.empty(n), "argmax": np.empty(n, np.int64), "lse": np.empty(n), "top2gap": np.empty(n),
            "tokens": np.empty(n, np.int64), "accept": np.empty(n, np.uint8),
            "selfcond": np.empty((n, d)) if want_selfcond else None}
+    if accept_mode == 1:
+        out["sample"], out["keygap"] = np.empty(n, np.int64), np.empty(n)
     for c in np.unique(rows // canvas_len):
         idx = np.nonzero(rows // canvas_len == c)[0]
         r = stage.step_rows(h_bits[rows[idx]], W_bits, E_bits, T, bound, int(seeds[c]), step, int(c),
-                            rows[idx] % canvas_len, vocab, want_selfcond)
+                            rows[idx] % canvas_len, vocab, want_selfcond, accept_mode=accept_mode)
         for k in out:
             if out[k] is not None:
                 out[k][idx] = r[k]
@@ -71,7 +76,12 @@ def compare(gpu, ora, rows, bound, check_selfcond=True, tag=""):
     assert bad.size == 0, f"{tag}: argmax mismatch at rows {rows[bad][:8]}"
     bad = np.nonzero(ok & (gpu["accept"][rows] != ora["accept"]))[0]
     assert bad.size == 0, f"{tag}: accept mismatch at rows {rows[bad][:8]}"
-    bad = np.nonzero(ok & (gpu["tokens"][rows] != ora["tokens"]))[0]
+    tok_ok = ok
+    if "keygap" in ora:
+        # sampled mode: an accepted position keeps the sample, decided by the key order
+        tok_ok = ok & ~((ora["accept"] == 1) & (ora["keygap"] < EXCL))
+        excl = excl | ((ora["accept"] == 1) & (ora["keygap"] < EXCL))
+    bad = np.nonzero(tok_ok & (gpu["tokens"][rows] != ora["tokens"]))[0]
     assert bad.size == 0, f"{tag}: token mismatch at rows {rows[bad][:8]}"
     dl = np.abs(gpu["lse"][rows] - ora["lse"])
     assert dl.max() <= 1e-3 * np.maximum(1.0, np.abs(ora["lse"])).max(), f"{tag}: lse error {dl.max():.3e}"
