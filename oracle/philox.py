@@ -16,9 +16,10 @@ Keying (a reading, the pages are silent): key = (lo32(seed), hi32(seed)) of the
 per-canvas seed; counter = (position i, step s, canvas c, tag).  Tags separate
 the streams: 0 canvas init, 1 re-noise, 2 stub target ids, 3 stub Gaussian noise.
 A token is word 0 mapped to [0, V) by the multiply-high floor(r * V / 2^32).
-The sampled-acceptance mode draws one word per (position, vocabulary entry):
-word (v mod 4) of counter (floor(v / 4), s, c, 4 + 256 i) - the fourth counter
-word is >= 4 there, so these streams never meet the four above.
+The sampled-acceptance mode draws one counter per (position, chunk of 64
+vocabulary entries): counter (floor(v / 64), s, c, 4 + 256 i), words 0 and 1 -
+the fourth counter word is >= 4 there, so these streams never meet the four
+above.
 
 Pins: known-answer vectors of the SC'11 reference implementation
 (tests/golden/philox4x32_10_kat.txt), bijectivity on a reduced counter set,
@@ -89,9 +90,11 @@ def uniform_token(seed, i, s, c, tag, vocab):
     return ((w0 * np.uint64(vocab)) >> np.uint64(32)).astype(np.int64)
 
 
-def vocab_words(seed, i, s, c, vocab):
-    """One 32-bit word per vocabulary entry v of position i: word (v mod 4) of counter
-    (floor(v / 4), s, c, TAG_SAMPLE + 256 i).  Returns uint32 [vocab] (vocab a multiple of 4)."""
-    q = np.arange(vocab // 4, dtype=np.uint64)
-    w = words(seed, q, s, c, TAG_SAMPLE + 256 * int(i))          # [vocab/4, 4]
-    return w.reshape(-1)
+
+def chunk_words(seed, i, s, c, n_chunks):
+    """Words 0 and 1 of counter (q, s, c, TAG_SAMPLE + 256 i) for every chunk q of position i.
+
+    Returns uint32 [n_chunks, 2]: word 0 drives the chunk's Gumbel key, word 1 the
+    draw inside the chunk."""
+    w = words(seed, np.arange(n_chunks, dtype=np.uint64), s, c, TAG_SAMPLE + 256 * int(i))
+    return w[:, :2]

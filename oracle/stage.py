@@ -18,7 +18,7 @@ Everything is float64 on the exact bf16 inputs the GPU receives (bf16 bit
 patterns widened to double).  The N x V logits block is formed explicitly: that
 is allowed here, and only here.
 
-The sampled-acceptance mode (``gumbel_noise``, ``gumbel_sample``; the accepted
+The sampled-acceptance mode (``gumbel_from_words``, ``gumbel_sample``; the accepted
 token is a draw from softmax(z / T) rather than the argmax) is a reading of the
 same passages - [DD] step 4 keeps "high-confidence" tokens and [JP] names
 temperature sharpening - that the pages leave open; the argmax mode stays the
@@ -119,41 +119,66 @@ def init_tokens(seed, c, vocab, n=256):
     return philox.uniform_token(seed, np.arange(n), 0, c, philox.TAG_INIT, vocab)
 
 
-def gumbel_noise(seed, i, s, c, vocab):
-    """Standard Gumbel noise g_v = -ln(-ln u_v) for every vocabulary entry of position i.
+SAMPLE_CHUNK = 64      # vocabulary entries per chunk of the sampled acceptance
 
-    u_v = (w_v + 1/2) / 2^32 with w_v from philox.vocab_words: uniform on (0, 1),
-    never 0 or 1.  -ln u_v is evaluated as -log1p(-(1 - u_v)), where
-    1 - u_v = (2^32 - 1 - w_v + 1/2) / 2^32 is exact in double, so the noise keeps
-    full relative precision as u_v -> 1 (where the winners of a large vocabulary lie).
-    """
-    w = philox.vocab_words(seed, i, s, c, vocab).astype(np.float64)
-    one_minus_u = (4294967295.0 - w + 0.5) / 4294967296.0
+
+def uniform_open(w):
+    """(u, 1 - u) for 32-bit words w: u = (w + 1/2) / 2^32 on (0, 1), both exact in double."""
+    w = np.asarray(w, np.float64)
+    return (w + 0.5) / 4294967296.0, (4294967295.0 - w + 0.5) / 4294967296.0
+
+
+def gumbel_from_words(w):
+    """Standard Gumbel noise g = -ln(-ln u), u from uniform_open; -ln u is taken as
+    -log1p(-(1 - u)), so the noise keeps full relative precision as u -> 1."""
+    _, one_minus_u = uniform_open(w)
     return -np.log(-np.log1p(-one_minus_u))
 
 
-def gumbel_sample(z, seed, s, c, positions):
-    """Sampled acceptance: a draw from softmax(z_i) for each row by the Gumbel-max trick.
+def gumbel_sample(z, seed, s, c, positions, chunk=SAMPLE_CHUNK):
+    """Sampled acceptance: an exact draw from softmax(z_i) for each row, in two levels.
 
-    The accepted token is argmax_v (z[i, v] + g[i, v]) (smallest v on an exact tie),
-    with g the per-(position, entry) Gumbel noise of gumbel_noise and z the
-    temperature-scaled logits (the distribution whose entropy the bound tests).
-    argmax of z + Gumbel noise is distributed as softmax(z) (Gumbel 1954; the
-    "Gumbel-max trick" of Maddison, Tarlow and Minka 2014).  Returns (sample int64 [n],
-    keygap float64 [n]: best key minus the second best, for the near-tie exclusion).
+    The vocabulary is cut into chunks of 64 consecutive entries.  (1) A chunk q is
+    chosen by the Gumbel-max trick on the chunk log-masses: argmax_q of
+    ln(sum_{v in q} e^{z_v}) + g_q (smallest q on a tie), g_q from word 0 of Philox
+    counter (q, s, c, 4 + 256 i) - so P(q) = mass_q / total (Gumbel 1954; the
+    "Gumbel-max trick", Maddison, Tarlow and Minka 2014).  (2) Inside it the entry
+    is the inverse CDF of the chunk's normalised probabilities at r = word 1 of the
+    same counter mapped by uniform_open: the smallest v whose running sum exceeds
+    r (the last entry with non-zero probability should rounding leave none).  The
+    two words are independent, so P(v) = P(q) P(v | q) = softmax(z)_v.
+    z are the temperature-scaled logits (the distribution whose entropy the bound
+    tests).  Returns (sample int64 [n], keygap [n]: best chunk key minus the
+    second best, cdf_margin [n]: min_k |running sum_k - r| in the chosen chunk),
+    the last two for the near-tie exclusions.
     """
     z = np.asarray(z, np.float64)
     n, V = z.shape
+    assert V % chunk == 0, "the vocabulary is a whole number of chunks"
+    nq = V // chunk
     out = np.empty(n, np.int64)
     gap = np.empty(n)
-    for r, i in enumerate(positions):
-        key = z[r] + gumbel_noise(seed, int(i), s, c, V)
-        b = int(np.argmax(key))
-        out[r] = b
+    margin = np.empty(n)
+    for row, i in enumerate(positions):
+        zc = z[row].reshape(nq, chunk)
+        mq = zc.max(axis=1)
+        with np.errstate(invalid="ignore"):
+            logmass = mq + np.log(np.exp(zc - mq[:, None]).sum(axis=1))
+        logmass = np.where(np.isfinite(mq), logmass, -np.inf)
+        w = philox.chunk_words(seed, int(i), s, c, nq)
+        key = logmass + gumbel_from_words(w[:, 0])
+        q = int(np.argmax(key))
         k2 = key.copy()
-        k2[b] = -np.inf
-        gap[r] = key[b] - k2.max() if V > 1 else np.inf
-    return out, gap
+        k2[q] = -np.inf
+        gap[row] = key[q] - k2.max() if nq > 1 else np.inf
+        r, _ = uniform_open(w[q, 1])
+        p = np.exp(zc[q] - logmass[q])
+        cs = np.cumsum(p)
+        hit = np.nonzero(cs > r)[0]
+        j = int(hit[0]) if hit.size else int(np.nonzero(p > 0)[0][-1])
+        out[row] = q * chunk + j
+        margin[row] = np.min(np.abs(cs - r))
+    return out, gap, margin
 
 
 def eb_accept(H, argmax, bound, renoise):
@@ -255,14 +280,14 @@ def step_rows(h_u16, W_u16, E_u16, T, bound, seed, s, c, positions, vocab, want_
     accept_mode 0 keeps the argmax at accepted positions, 1 a Gumbel-max sample of
     softmax(z / T) (gumbel_sample).
     Returns dict with H, argmax, lse, top2gap, tokens, accept, selfcond, and with
-    accept_mode 1 also sample and keygap.
+    accept_mode 1 also sample, keygap and cdf_margin.
     """
     h = bf16_to_f64(h_u16)
     z = logits_chunked(h, W_u16, T)
     out = {}
     kept = None
     if accept_mode == 1:
-        out["sample"], out["keygap"] = gumbel_sample(z, seed, s, c, positions)
+        out["sample"], out["keygap"], out["cdf_margin"] = gumbel_sample(z, seed, s, c, positions)
         kept = out["sample"]
     st = distribution_stats(z)
     del z
