@@ -29,6 +29,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 V, D, N_POS, STEP, BOUND = 262144, 2816, 256, 1, 0.1
+ACCEPT_MODE = 0            # 0: accepted positions keep the argmax; 1: a Gumbel-max sample (--accept sample)
 METRIC = "canvas positions/s per denoise step (V=262144,d=2816); % of roofline"
 WORKLOAD = ("single-step microbenchmark: 1 canvas of 256 positions, V=262144, d=2816, tied bf16 E=W ~N(0,0.02), "
             "hidden bf16 N(0,1)/sqrt(d)*8, step 1 (T=0.8), bound 0.1; outputs tokens/H/argmax/accept/self-cond fp32")
@@ -177,6 +178,14 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- CPU oracle leg
+def _set_accept(mode):
+    """--accept sample: time the sampled-acceptance kernel instead of the argmax one."""
+    global ACCEPT_MODE, WORKLOAD
+    ACCEPT_MODE = mode
+    if mode == 1:
+        WORKLOAD = WORKLOAD.replace("bound 0.1;", "bound 0.1, accepted tokens drawn by Gumbel-max sampling;")
+
+
 def oracle_sample_rate(W64, h_bits, n_rows, T):
     """Time the float64 oracle on n_rows positions of the workload; returns (positions/s, seconds, threads).
 
@@ -189,7 +198,7 @@ def oracle_sample_rate(W64, h_bits, n_rows, T):
     except Exception:
         threads = os.cpu_count() or 1
     t0 = time.perf_counter()
-    stage.step_rows(h_bits[:n_rows], W64, W64, T, BOUND, 0, STEP, 0, list(range(n_rows)), V)
+    stage.step_rows(h_bits[:n_rows], W64, W64, T, BOUND, 0, STEP, 0, list(range(n_rows)), V, accept_mode=ACCEPT_MODE)
     dt = time.perf_counter() - t0
     return n_rows / dt, dt, threads
 
@@ -247,7 +256,7 @@ def run_gpu(args):
 
     # replicas: every rank owns one canvas of its own (seed = its global canvas index)
     c0, _ = shard_canvases(world, rank, world)
-    p = dg.params(1, V, D)
+    p = dg.params(1, V, D, accept_mode=ACCEPT_MODE)
     W = synth.weights(V, D, seed=1234).to(dev)
     h_host = synth.gaussian_hidden(N_POS, D, seed=42)
     ws = dg.Workspace(p, dev)
@@ -327,7 +336,7 @@ def run_gpu(args):
         peak_tf_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
         achieved = FLOPS_PER_STEP / (k1_max * 1e-3) / 1e12
         roof_ms = max(FLOPS_PER_STEP / (peak_tf * 1e12), WE_BYTES_PER_STEP / (float(peaks.get("hbm_gbs", 6650.0)) * 1e9)) * 1e3
-        traffic = profiled_traffic()
+        traffic = profiled_traffic() if ACCEPT_MODE == 0 else None    # the profile is of the argmax kernel
         value = world * N_POS / (ms_per_step * 1e-3)
         line = {
             "metric": METRIC, "value": value, "unit": "positions/s", "n_gpus": world, "steps": args.steps,
@@ -340,7 +349,8 @@ def run_gpu(args):
             "steps_per_s": 1e3 / ms_per_step,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": achieved / peak_tf, "traffic": traffic,
-                         "kernel": "dg_fused_kernel", "kernel_ms": k1_max, "launches_timed": n_k1,
+                         "kernel": "dg_fused_sample_kernel" if ACCEPT_MODE else "dg_fused_kernel",
+                         "kernel_ms": k1_max, "launches_timed": n_k1,
                          "flops_per_launch": FLOPS_PER_STEP, "peak_source": f"{peaks_src} bf16 burst",
                          "frac_of_sustained": achieved / peak_tf_sus,
                          "step_frac": roof_ms / ms_per_step, "roofline_step_ms": roof_ms},
@@ -375,11 +385,14 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-rows", type=int, default=256, help="positions in the oracle's bounded CPU sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--accept", choices=["argmax", "sample"], default="argmax",
+                    help="token kept at accepted positions (sample: Gumbel-max draw from softmax(z/T))")
     ap.add_argument("--vocab", type=int, default=262144,
                     help="vocabulary size; smaller values are for profiler captures only, not bench lines")
     args = ap.parse_args(argv)
     if args.vocab != V:
         _set_vocab(args.vocab)
+    _set_accept(1 if args.accept == "sample" else 0)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":

@@ -59,7 +59,7 @@ __host__ __device__ inline int32_t philox_token(uint64_t seed, uint32_t i, uint3
 }
 
 enum : uint32_t { kTagInit = 0, kTagRenoise = 1, kTagStubTarget = 2, kTagStubNoise = 3 };
-// sampled acceptance: counter (v / 4, step, canvas, kTagSample + 256 i), one word per entry v
+// sampled acceptance: counter (v / 64, step, canvas, kTagSample + 256 i), one per 64-entry chunk
 constexpr uint32_t kTagSample = 4;
 
 // ------------------------------------------------------------------ plan and layout

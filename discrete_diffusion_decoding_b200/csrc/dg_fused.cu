@@ -155,17 +155,15 @@ struct Schedule {
 
 }  // namespace
 
-// Gumbel-max key of one logit, in log2 units up to a constant: s log2(e)/T - log2(-log2 u)
-// with u = 1 - eps, eps = (~w + 1/2) 2^-32 (u = (w + 1/2) 2^-32 exactly), so that
-// argmax_v key = argmax_v (z_v + g_v) with g = -ln(-ln u) standard Gumbel noise.
-// -log2(1 - eps) comes from the SFU logarithm, or below eps = 2^-8 from its series
-// log2(e) (eps + eps^2/2 + eps^3/3) (relative truncation error < 2^-26), which keeps
-// full precision where u -> 1, the region the winners of a large vocabulary come from.
-__device__ __forceinline__ float gumbel_key(float s, float c2, uint32_t w) {
+// -log2(u) for u = (w + 1/2) 2^-32, from eps = 1 - u = (~w + 1/2) 2^-32: the SFU
+// logarithm of 1 - eps, or below eps = 2^-8 the series log2(e) (eps + eps^2/2 + eps^3/3)
+// (relative truncation error < 2^-26), which keeps full precision as u -> 1.  Then
+// -log2(-log2 u) is the standard Gumbel variable g = -ln(-ln u) in log2 units, up to
+// the constant log2(log2 e).
+__device__ __forceinline__ float neg_log2_uniform(uint32_t w) {
     const float eps = fmaf(static_cast<float>(~w), 2.3283064365386963e-10f, 1.1641532182693481e-10f);
     const float series = eps * fmaf(eps, fmaf(eps, 0.333333343f, 0.5f), 1.0f) * 1.44269502f;
-    const float e2 = eps < 0.00390625f ? series : -fast_log2(1.0f - eps);
-    return fmaf(s, c2, -fast_log2(e2));
+    return eps < 0.00390625f ? series : -fast_log2(1.0f - eps);
 }
 
 template <bool kSample>
@@ -506,6 +504,7 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                     for (int c0 = 0; c0 < kBV; c0 += 64) {
                         uint32_t v[64];
                         tmem_ld64(tmem + kTmemS + lane_addr + c0, v);
+                        float lc = 0.f;            // this 64-entry chunk's mass, relative to m_ref
 #pragma unroll
                         for (int i = 0; i < 64; i += 2) {
                             const float s0 = __uint_as_float(v[i]), s1 = __uint_as_float(v[i + 1]);
@@ -513,26 +512,37 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                             if (s1 > best) { best = s1; best_idx = v0 + c0 + i + 1; }
                             const float y0 = fmaf(s0, c2, -m_ref), y1 = fmaf(s1, c2, -m_ref);
                             const float e0 = fast_exp2(y0), e1 = fast_exp2(y1);
-                            l += e0 + e1;
+                            lc += e0 + e1;
                             u = fmaf(e0, y0, fmaf(e1, y1, u));
                             const float recv = __shfl_xor_sync(0xffffffffu, odd ? e0 : e1, 1);
                             const int col = c0 + i + (odd ? 1 : 0);
                             *reinterpret_cast<uint32_t*>(pt + static_cast<size_t>(col) * kCanvas + prow) =
                                 pack_bf16(odd ? recv : e0, odd ? e1 : recv);
                         }
+                        l += lc;
                         if constexpr (kSample) {
-                            // Gumbel-max over the same logits: word (v mod 4) of Philox counter
-                            // (v / 4, step, canvas, 4 + 256 i); strict > keeps the smallest v on a tie
+                            // two-level draw: the chunk's Gumbel-max key on its log-mass (word 0 of
+                            // Philox counter (v / 64, step, canvas, 4 + 256 i)), absolute in log2
+                            // units; strict > keeps the smallest chunk on a tie.  A chunk that takes
+                            // the lead picks its entry by the inverse CDF at word 1.
+                            const uint32_t q = static_cast<uint32_t>(v0 + c0) >> 6;
+                            uint32_t w[4] = {q, static_cast<uint32_t>(a.step), canvas, pos_word};
+                            philox4x32_10(w, key_lo, key_hi);
+                            const float kq = (m_ref + fast_log2(lc)) - fast_log2(neg_log2_uniform(w[0]));
+                            if (kq > skey) {
+                                skey = kq;
+                                const float target = fmaf(static_cast<float>(w[1]), 2.3283064365386963e-10f,
+                                                          1.1641532182693481e-10f) * lc;
+                                float run = 0.f;
+                                int pick = -1, last = 0;
 #pragma unroll
-                            for (int i = 0; i < 64; i += 4) {
-                                const uint32_t v4 = static_cast<uint32_t>(v0 + c0 + i);
-                                uint32_t w[4] = {v4 >> 2, static_cast<uint32_t>(a.step), canvas, pos_word};
-                                philox4x32_10(w, key_lo, key_hi);
-#pragma unroll
-                                for (int j = 0; j < 4; ++j) {
-                                    const float kj = gumbel_key(__uint_as_float(v[i + j]), c2, w[j]);
-                                    if (kj > skey) { skey = kj; sidx = static_cast<int>(v4) + j; }
+                                for (int i = 0; i < 64; ++i) {
+                                    const float e = fast_exp2(fmaf(__uint_as_float(v[i]), c2, -m_ref));
+                                    run += e;
+                                    if (pick < 0 && run > target) pick = i;
+                                    if (e > 0.f) last = i;
                                 }
+                                sidx = v0 + c0 + (pick >= 0 ? pick : last);
                             }
                         }
                     }

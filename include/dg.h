@@ -79,14 +79,17 @@ typedef struct {
     int group;          /* column-slice group size of the fused kernel; 0 = automatic */
     int accept_mode;    /* token kept at an accepted position (H <= eb_bound):
                          *   0 = the argmax (default);
-                         *   1 = a draw from softmax(z / T_s) by the Gumbel-max trick: the argmax
-                         *       over v of z[i,v] + g[i,v], g = -ln(-ln u), u = (w + 1/2) / 2^32,
-                         *       w = word (v mod 4) of Philox4x32-10 counter
-                         *       (v / 4, step, canvas, 4 + 256 i) under the canvas seed; smallest
-                         *       v on a tie.  The pages leave open whether the kept token is the
-                         *       most likely one or a sample (deep dive, reverse diffusion step 4;
-                         *       juhoplayground overview, logits scheduler); argmax, entropy, LSE
-                         *       and the self-conditioning vector are the same in both modes. */
+                         *   1 = an exact draw from softmax(z / T_s) in two levels: the 64-entry
+                         *       chunk q = v / 64 with the largest ln(sum_{v in q} e^{z[i,v]}) + g_q
+                         *       (g = -ln(-ln u), u = (w0 + 1/2) / 2^32; smallest q on a tie), then
+                         *       the inverse CDF of the chunk's normalised probabilities at
+                         *       r = (w1 + 1/2) / 2^32; w0, w1 = words 0, 1 of Philox4x32-10
+                         *       counter (q, step, canvas, 4 + 256 i) under the canvas seed (the
+                         *       Gumbel-max trick on chunk masses).
+                         *   The pages leave open whether the kept token is the most likely one
+                         *   or a sample (deep dive, reverse diffusion step 4; juhoplayground
+                         *   overview, logits scheduler); argmax, entropy, LSE and the
+                         *   self-conditioning vector are the same in both modes. */
 } dg_params;
 
 /* Fill a dg_params with the pages' defaults for C canvases of a (V, d) head. */

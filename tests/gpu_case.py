@@ -5,8 +5,9 @@ Tolerances (per position): H within 1e-3 nats; self-conditioning within 2e-2
 relative L2; tokens, accept flags and argmax bit-exact except at positions whose
 oracle entropy is within 1e-3 of the bound or whose top-2 logits (z = h.W/T)
 differ by less than 1e-3 - those are listed and excluded.  In the sampled
-acceptance mode the kept token is the Gumbel-max sample; positions whose two
-best keys (z + g) differ by less than 1e-3 are excluded the same way.
+acceptance mode the kept token is the two-level sample; positions whose two best
+chunk keys differ by less than 1e-3, or whose in-chunk running probability passes
+within 1e-4 of the uniform draw, are excluded the same way.
 """
 
 import numpy as np
@@ -53,7 +54,7 @@ def oracle_rows(h_bits, W_bits, E_bits, T, bound, seeds, step, rows, vocab, canv
            "tokens": np.empty(n, np.int64), "accept": np.empty(n, np.uint8),
            "selfcond": np.empty((n, d)) if want_selfcond else None}
     if accept_mode == 1:
-        out["sample"], out["keygap"] = np.empty(n, np.int64), np.empty(n)
+        out["sample"], out["keygap"], out["cdf_margin"] = np.empty(n, np.int64), np.empty(n), np.empty(n)
     for c in np.unique(rows // canvas_len):
         idx = np.nonzero(rows // canvas_len == c)[0]
         r = stage.step_rows(h_bits[rows[idx]], W_bits, E_bits, T, bound, int(seeds[c]), step, int(c),
@@ -79,8 +80,9 @@ def compare(gpu, ora, rows, bound, check_selfcond=True, tag=""):
     tok_ok = ok
     if "keygap" in ora:
         # sampled mode: an accepted position keeps the sample, decided by the key order
-        tok_ok = ok & ~((ora["accept"] == 1) & (ora["keygap"] < EXCL))
-        excl = excl | ((ora["accept"] == 1) & (ora["keygap"] < EXCL))
+        near = (ora["accept"] == 1) & ((ora["keygap"] < EXCL) | (ora["cdf_margin"] < 1e-4))
+        tok_ok = ok & ~near
+        excl = excl | near
     bad = np.nonzero(tok_ok & (gpu["tokens"][rows] != ora["tokens"]))[0]
     assert bad.size == 0, f"{tag}: token mismatch at rows {rows[bad][:8]}"
     dl = np.abs(gpu["lse"][rows] - ora["lse"])
