@@ -21,7 +21,7 @@ from . import stage
 
 def decode_batch(W_u16, E_u16, seeds, hidden, vocab, max_steps=48, t_start=0.8, t_end=0.4,
                  bound=0.1, stop_thresh=0.005, stability=2, canvas_len=256,
-                 want_selfcond=False, record=False):
+                 want_selfcond=False, record=False, accept_rule=0):
     """Free-running decode of C independent canvases in one batch.
 
     hidden(tokens_of_canvas[int64 canvas_len], s, c) -> bf16 bits [canvas_len, d].
@@ -44,7 +44,7 @@ def decode_batch(W_u16, E_u16, seeds, hidden, vocab, max_steps=48, t_start=0.8, 
                 continue
             h = hidden(tokens[c].copy(), s, c)
             r = stage.denoise_step(h, W_u16, E_u16, T, bound, [seeds[c]], s, vocab,
-                                   canvas_len, want_selfcond, canvas_ids=[c])
+                                   canvas_len, want_selfcond, canvas_ids=[c], accept_rule=accept_rule)
             tok, acc = r["tokens"], r["accept"]
             stable[c], stop = stage.stop_update(r["mean_H"][0], r["argmax"], prev[c], stable[c], s,
                                                 stop_thresh, stability)
@@ -52,7 +52,8 @@ def decode_batch(W_u16, E_u16, seeds, hidden, vocab, max_steps=48, t_start=0.8, 
             if record:
                 rec["canvases"][c] = {"h": h, "H": r["H"], "argmax": r["argmax"], "tokens_in": tokens[c].copy(),
                                       "tokens": tok, "accept": acc, "mean_H": r["mean_H"][0],
-                                      "stable": stable[c], "stop": stop, "top2gap": r["top2gap"]}
+                                      "stable": stable[c], "stop": stop, "top2gap": r["top2gap"],
+                                      "cut_margin": r["cut_margin"], "order_gap": r["order_gap"]}
             tokens[c] = tok
             if stop or s == max_steps:
                 stopped[c] = True

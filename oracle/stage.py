@@ -192,6 +192,37 @@ def eb_accept(H, argmax, bound, renoise):
     return tokens, acc.astype(np.uint8)
 
 
+def group_accept(H, kept, bound, renoise):
+    """Group entropy-bounded accept for the positions of one canvas ([JP] sampler: token
+    groups are accepted by entropy-based confidence; [DD] settings table: bound 0.1).
+
+    Reading: order the positions by entropy max(H, 0), ties by position, and accept the
+    longest prefix whose cumulative entropy is <= bound - the largest set of positions
+    whose entropies sum to at most the bound, and of the sets of that size the one with
+    the least total; the other positions take their re-noise draw.  No position is
+    forced through when even the smallest entropy exceeds the bound (as in the
+    per-position rule).  kept is the token an accepted position keeps (the argmax, or
+    the sample of the sampled mode).
+    Returns (tokens, accept uint8, cut_margin, order_gap): the distance from the bound
+    of the cumulative sums on either side of the cut, and the entropy gap between the
+    last accepted and the first rejected position (for the parity exclusions).
+    """
+    H = np.maximum(np.asarray(H, np.float64), 0.0)
+    n = H.size
+    order = np.lexsort((np.arange(n), H))
+    S = np.cumsum(H[order])
+    k = int(np.count_nonzero(S <= bound))          # S is non-decreasing: the accepted prefix
+    acc = np.zeros(n, bool)
+    acc[order[:k]] = True
+    tokens = np.where(acc, kept, renoise).astype(np.int64)
+    cut = [abs(S[k - 1] - bound)] if k > 0 else []
+    if k < n:
+        cut.append(abs(S[k] - bound))
+    cut_margin = min(cut) if cut else np.inf
+    order_gap = H[order[k]] - H[order[k - 1]] if 0 < k < n else np.inf
+    return tokens, acc.astype(np.uint8), float(cut_margin), float(order_gap)
+
+
 def stop_update(mean_H, argmax, prev_argmax, stable, s, stop_thresh=0.005, stability=2):
     """Two-fold adaptive stop for one canvas ([DD] conditions 1 and 2).
 
@@ -207,27 +238,35 @@ def stop_update(mean_H, argmax, prev_argmax, stable, s, stop_thresh=0.005, stabi
 
 
 def denoise_step(h_u16, W_u16, E_u16, T, bound, seeds, s, vocab, canvas_len=256,
-                 want_selfcond=True, canvas_ids=None):
+                 want_selfcond=True, canvas_ids=None, accept_rule=0):
     """One step over all canvases of a batch, from bf16 bit patterns.
 
     h_u16 [N, d], W_u16 / E_u16 [V, d] (uint16 bf16 bits, or their exact float64
     widening), seeds [C] (uint64),
     N = C * canvas_len; canvas_ids[c] (default c) is the canvas word of the
-    Philox counter.  Returns dict with H, argmax, lse, top2gap, tokens,
-    accept, selfcond (or None), mean_H per canvas.
+    Philox counter.  accept_rule 0 accepts per position (eb_accept), 1 by groups
+    (group_accept; the cut margins are returned as cut_margin / order_gap per canvas).
+    Returns dict with H, argmax, lse, top2gap, tokens, accept, selfcond (or None),
+    mean_H per canvas.
     """
     h = bf16_to_f64(h_u16)
     W = _widen(np.asarray(W_u16))
     E = W if E_u16 is W_u16 else _widen(np.asarray(E_u16))
     n = h.shape[0]
     C = n // canvas_len
-    out = {k: [] for k in ("H", "argmax", "lse", "top2gap", "tokens", "accept", "selfcond", "max")}
+    out = {k: [] for k in ("H", "argmax", "lse", "top2gap", "tokens", "accept", "selfcond", "max",
+                           "cut_margin", "order_gap")}
     for c in range(C):
         sl = slice(c * canvas_len, (c + 1) * canvas_len)
         st = distribution_stats(logits(h[sl], W, T))
         cid = c if canvas_ids is None else int(canvas_ids[c])
         ren = renoise_tokens(int(seeds[c]), s, cid, vocab, canvas_len)
-        tok, acc = eb_accept(st["H"], st["argmax"], bound, ren)
+        if accept_rule == 1:
+            tok, acc, cm, og = group_accept(st["H"], st["argmax"], bound, ren)
+            out["cut_margin"].append(np.array([cm]))
+            out["order_gap"].append(np.array([og]))
+        else:
+            tok, acc = eb_accept(st["H"], st["argmax"], bound, ren)
         out["H"].append(st["H"])
         out["argmax"].append(st["argmax"])
         out["lse"].append(st["lse"])
