@@ -30,6 +30,7 @@ if ROOT not in sys.path:
 
 V, D, N_POS, STEP, BOUND = 262144, 2816, 256, 1, 0.1
 ACCEPT_MODE = 0            # 0: accepted positions keep the argmax; 1: a Gumbel-max sample (--accept sample)
+ACCEPT_RULE = 0            # 0: accept every position with H <= bound; 1: by groups (--rule group)
 METRIC = "canvas positions/s per denoise step (V=262144,d=2816); % of roofline"
 WORKLOAD = ("single-step microbenchmark: 1 canvas of 256 positions, V=262144, d=2816, tied bf16 E=W ~N(0,0.02), "
             "hidden bf16 N(0,1)/sqrt(d)*8, step 1 (T=0.8), bound 0.1; outputs tokens/H/argmax/accept/self-cond fp32")
@@ -178,12 +179,14 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- CPU oracle leg
-def _set_accept(mode):
-    """--accept sample: time the sampled-acceptance kernel instead of the argmax one."""
-    global ACCEPT_MODE, WORKLOAD
-    ACCEPT_MODE = mode
+def _set_accept(mode, rule=0):
+    """--accept sample / --rule group: time the sampled-acceptance kernel or the group rule."""
+    global ACCEPT_MODE, ACCEPT_RULE, WORKLOAD
+    ACCEPT_MODE, ACCEPT_RULE = mode, rule
     if mode == 1:
-        WORKLOAD = WORKLOAD.replace("bound 0.1;", "bound 0.1, accepted tokens drawn by Gumbel-max sampling;")
+        WORKLOAD = WORKLOAD.replace("bound 0.1", "bound 0.1, accepted tokens drawn by Gumbel-max sampling")
+    if rule == 1:
+        WORKLOAD = WORKLOAD.replace("bound 0.1", "bound 0.1 on the cumulative entropy of each canvas's accepted group")
 
 
 def oracle_sample_rate(W64, h_bits, n_rows, T):
@@ -198,7 +201,12 @@ def oracle_sample_rate(W64, h_bits, n_rows, T):
     except Exception:
         threads = os.cpu_count() or 1
     t0 = time.perf_counter()
-    stage.step_rows(h_bits[:n_rows], W64, W64, T, BOUND, 0, STEP, 0, list(range(n_rows)), V, accept_mode=ACCEPT_MODE)
+    r = stage.step_rows(h_bits[:n_rows], W64, W64, T, BOUND, 0, STEP, 0, list(range(n_rows)), V,
+                        accept_mode=ACCEPT_MODE)
+    if ACCEPT_RULE == 1:
+        # the group rule needs every position of the canvas; a partial sample ranks what it has
+        kept = r["sample"] if ACCEPT_MODE == 1 else r["argmax"]
+        stage.group_accept(r["H"], kept, BOUND, r["tokens"])
     dt = time.perf_counter() - t0
     return n_rows / dt, dt, threads
 
@@ -256,7 +264,7 @@ def run_gpu(args):
 
     # replicas: every rank owns one canvas of its own (seed = its global canvas index)
     c0, _ = shard_canvases(world, rank, world)
-    p = dg.params(1, V, D, accept_mode=ACCEPT_MODE)
+    p = dg.params(1, V, D, accept_mode=ACCEPT_MODE, accept_rule=ACCEPT_RULE)
     W = synth.weights(V, D, seed=1234).to(dev)
     h_host = synth.gaussian_hidden(N_POS, D, seed=42)
     ws = dg.Workspace(p, dev)
@@ -387,12 +395,14 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--accept", choices=["argmax", "sample"], default="argmax",
                     help="token kept at accepted positions (sample: Gumbel-max draw from softmax(z/T))")
+    ap.add_argument("--rule", choices=["position", "group"], default="position",
+                    help="accepted positions: H <= bound each, or the canvas's entropy-ordered group within the bound")
     ap.add_argument("--vocab", type=int, default=262144,
                     help="vocabulary size; smaller values are for profiler captures only, not bench lines")
     args = ap.parse_args(argv)
     if args.vocab != V:
         _set_vocab(args.vocab)
-    _set_accept(1 if args.accept == "sample" else 0)
+    _set_accept(1 if args.accept == "sample" else 0, 1 if args.rule == "group" else 0)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":

@@ -19,7 +19,7 @@ class DgParams(ctypes.Structure):
                 ("hidden", ctypes.c_int), ("max_steps", ctypes.c_int), ("t_start", ctypes.c_float),
                 ("t_end", ctypes.c_float), ("eb_bound", ctypes.c_float), ("stop_thresh", ctypes.c_float),
                 ("stability", ctypes.c_int), ("tied", ctypes.c_int), ("group", ctypes.c_int),
-                ("accept_mode", ctypes.c_int)]
+                ("accept_mode", ctypes.c_int), ("accept_rule", ctypes.c_int)]
 
 
 class DgError(RuntimeError):

@@ -112,6 +112,7 @@ bool params_ok(const dg_params* p) {
     if (!(p->t_start > 0.f) || !(p->t_end > 0.f)) return false;
     if (p->stability < 0) return false;
     if (p->accept_mode != 0 && p->accept_mode != 1) return false;
+    if (p->accept_rule != 0 && p->accept_rule != 1) return false;
     return true;
 }
 
@@ -197,6 +198,7 @@ void dg_params_default(dg_params* p, int n_canvas, int vocab, int hidden) {
     p->tied = 1;
     p->group = 0;
     p->accept_mode = 0;
+    p->accept_rule = 0;
 }
 
 float dg_temperature(const dg_params* p, int step) {
@@ -350,6 +352,8 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
     ca.skey = fa.skey;
     ca.sidx = fa.sidx;
     ca.accept_mode = p->accept_mode;
+    ca.accept_rule = p->accept_rule;
+    ca.kept = at<int32_t>(workspace_dev, L.kept);
     ca.opart = fa.opart;
     ca.entropy = entropy_dev;
     ca.argmax = argmax_dev;
@@ -370,9 +374,10 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
     dg_combine_kernel<<<combine_grid(pl.N, pl.d), 256, 0, s>>>(ca);
     if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
 
+    GroupAcceptArgs ga{p->accept_rule, p->eb_bound, ca.kept, seeds_dev, tokens_dev, accept_dev, pl.V};
     dg_stop_kernel<<<pl.C, kCanvas, 0, s>>>(entropy_dev, argmax_dev, at<int32_t>(workspace_dev, L.prev_argmax),
                                             at<int32_t>(workspace_dev, L.stable), stop, p->stop_thresh, p->stability,
-                                            step);
+                                            step, ga);
     if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
     g_last_launches = 3;
     return DG_OK;

@@ -82,6 +82,7 @@ struct Layout {
     size_t stat_idx;                              // [n_slots][G][256] int32
     size_t skey;                                  // [n_slots][G][256] float: best Gumbel-max key (sampled mode)
     size_t sidx;                                  // [n_slots][G][256] int32: its vocabulary index
+    size_t kept;                                  // [N] int32: token an accepted position keeps (group rule)
     size_t opart;                                 // [n_slots][256][d] float
     size_t total;
 };
@@ -107,6 +108,7 @@ inline Layout make_layout(const Plan& pl) {
     L.stat_idx = take(sizeof(int32_t) * static_cast<size_t>(pl.n_slots) * pl.group * kCanvas);
     L.skey = take(sizeof(float) * static_cast<size_t>(pl.n_slots) * pl.group * kCanvas);
     L.sidx = take(sizeof(int32_t) * static_cast<size_t>(pl.n_slots) * pl.group * kCanvas);
+    L.kept = take(sizeof(int32_t) * pl.N);
     L.opart = take(sizeof(float) * static_cast<size_t>(pl.n_slots) * kCanvas * pl.d);
     L.total = o;
     return L;

@@ -744,7 +744,9 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
                 a.entropy[n] = H;
                 a.argmax[n] = bidx;
                 if (a.lse) a.lse[n] = ln2 * (M + log2f(L));
-                if (a.tokens) {
+                if (a.tokens && a.accept_rule == 1) {
+                    a.kept[n] = a.accept_mode == 1 ? sidx : bidx;     // accepted by groups in dg_stop_kernel
+                } else if (a.tokens) {
                     const bool acc = H <= a.bound;
                     a.tokens[n] = acc ? (a.accept_mode == 1 ? sidx : bidx)
                                       : philox_token(a.seeds[c], static_cast<uint32_t>(crow),

@@ -44,6 +44,8 @@ struct CombineArgs {
     const float* skey;       // sampled acceptance: Gumbel-max keys / indices (accept_mode 1)
     const int32_t* sidx;
     int accept_mode;         // 0: keep the argmax, 1: keep the Gumbel-max sample
+    int accept_rule;         // 0: accept per position here; 1: only store the kept token (group rule)
+    int32_t* kept;           // [N] the kept token of every position (accept_rule 1)
     const float* opart;
     float* entropy;
     int32_t* argmax;
@@ -69,8 +71,20 @@ __global__ void dg_combine_kernel(const CombineArgs a);
 // small kernels (dg_small.cu)
 __global__ void dg_init_kernel(const uint64_t* seeds, int32_t* tokens, int32_t* prev_argmax, int32_t* stable,
                                int32_t* stop, int32_t* err, uint32_t* counters, int n_counter_words, int C, int V);
+// Group entropy-bounded accept, applied by dg_stop_kernel before the stop reduction
+// when `rule` is 1 (nothing happens with rule 0 or a null tokens pointer).
+struct GroupAcceptArgs {
+    int rule;
+    float bound;
+    const int32_t* kept;
+    const uint64_t* seeds;
+    int32_t* tokens;
+    uint8_t* accept;
+    int V;
+};
+
 __global__ void dg_stop_kernel(const float* entropy, const int32_t* argmax, int32_t* prev_argmax, int32_t* stable,
-                               int32_t* stop, float stop_thresh, int stability, int step);
+                               int32_t* stop, float stop_thresh, int stability, int step, GroupAcceptArgs ga);
 __global__ void dg_stub_kernel(const uint64_t* seeds, const __nv_bfloat16* E, const int32_t* tokens,
                                const int32_t* stop, __nv_bfloat16* h, float a_s, float gain, float noise, int step,
                                int d, int V, int N);

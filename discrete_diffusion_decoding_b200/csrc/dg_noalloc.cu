@@ -200,6 +200,8 @@ extern "C" dg_status dg_denoise_stats_noalloc(const dg_params* p, int step, cons
     ca.skey = nullptr;          // statistics only: no acceptance, so no sample
     ca.sidx = nullptr;
     ca.accept_mode = 0;
+    ca.accept_rule = 0;
+    ca.kept = nullptr;
     ca.opart = fa.opart;
     ca.entropy = entropy_dev;
     ca.argmax = argmax_dev;

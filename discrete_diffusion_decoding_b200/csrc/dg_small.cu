@@ -30,15 +30,64 @@ __global__ void dg_init_kernel(const uint64_t* seeds, int32_t* tokens, int32_t* 
     for (int w = n; w < n_counter_words; w += gridDim.x * blockDim.x) counters[w] = 0u;
 }
 
+// Group entropy-bounded accept of one canvas (juhoplayground overview, entropy
+// bounded sampler: token groups are accepted by entropy; deep dive bound 0.1):
+// the positions ordered by (max(H, 0), position) - a bitonic sort of 64-bit keys
+// (entropy bits, position), monotone because the entropy is non-negative - and the
+// longest prefix whose cumulative entropy is <= bound keeps its token; the other
+// positions take the uniform re-noise draw (Philox tag 1, this step).  The
+// cumulative sum runs in sorted order in one thread.
+__device__ void group_accept(const float* entropy, const GroupAcceptArgs& ga, int c, int step) {
+    __shared__ unsigned long long key[kCanvas];
+    __shared__ int n_acc;
+    const int tid = threadIdx.x;
+    const float h = fmaxf(entropy[c * kCanvas + tid], 0.f);
+    key[tid] = (static_cast<unsigned long long>(__float_as_uint(h)) << 32) | static_cast<unsigned>(tid);
+    __syncthreads();
+    for (int k = 2; k <= kCanvas; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const int p = tid ^ j;
+            if (p > tid) {
+                const unsigned long long x = key[tid], y = key[p];
+                const bool up = (tid & k) == 0;
+                if ((x > y) == up) {
+                    key[tid] = y;
+                    key[p] = x;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    if (tid == 0) {
+        float S = 0.f;
+        int k = 0;
+        for (; k < kCanvas; ++k) {
+            S += __uint_as_float(static_cast<uint32_t>(key[k] >> 32));
+            if (!(S <= ga.bound)) break;
+        }
+        n_acc = k;
+    }
+    __syncthreads();
+    const int i = static_cast<int>(key[tid] & 0xffffffffu);      // the position of sorted rank tid
+    const int n = c * kCanvas + i;
+    const bool acc = tid < n_acc;
+    ga.tokens[n] = acc ? ga.kept[n]
+                       : philox_token(ga.seeds[c], static_cast<uint32_t>(i), static_cast<uint32_t>(step),
+                                      static_cast<uint32_t>(c), kTagRenoise, static_cast<uint32_t>(ga.V));
+    ga.accept[n] = acc ? 1 : 0;
+}
+
 // Two-fold adaptive stop (deep dive, "Two-Fold Adaptive Stopping"): one CTA of
 // 256 threads per canvas; the mean entropy is a fixed-order tree sum; the
 // stable counter grows while the argmax vector repeats (0 at step 1) and resets
-// on any change; stop = mean H < threshold AND stable >= stability.
+// on any change; stop = mean H < threshold AND stable >= stability.  With the
+// group rule the canvas's accept / re-noise runs first (group_accept).
 __global__ void __launch_bounds__(256) dg_stop_kernel(const float* entropy, const int32_t* argmax,
                                                       int32_t* prev_argmax, int32_t* stable, int32_t* stop,
-                                                      float stop_thresh, int stability, int step) {
+                                                      float stop_thresh, int stability, int step, GroupAcceptArgs ga) {
     const int c = blockIdx.x;
     if (stop[c]) return;
+    if (ga.rule == 1 && ga.tokens != nullptr) group_accept(entropy, ga, c, step);
     const int tid = threadIdx.x;
     const int n = c * kCanvas + tid;
     float h = entropy[n];

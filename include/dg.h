@@ -90,6 +90,13 @@ typedef struct {
                          *   or a sample (deep dive, reverse diffusion step 4; juhoplayground
                          *   overview, logits scheduler); argmax, entropy, LSE and the
                          *   self-conditioning vector are the same in both modes. */
+    int accept_rule;    /* which positions are accepted:
+                         *   0 = every position with H <= eb_bound (default);
+                         *   1 = by groups: the canvas's positions ordered by max(H, 0) (ties by
+                         *       position) and the longest prefix whose cumulative entropy is
+                         *       <= eb_bound - the sampler accepting token groups by entropy
+                         *       (juhoplayground overview, entropy bounded sampler).  No position
+                         *       is forced through.  Applied in the per-canvas stop kernel. */
 } dg_params;
 
 /* Fill a dg_params with the pages' defaults for C canvases of a (V, d) head. */
