@@ -117,20 +117,23 @@ def profiled_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms; summary() keeps the samples
+    whose timestamps fall inside the timed region (the sampler is started before the warm-up
+    so that its start-up does not eat into the region)."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index):
+        import tempfile
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        fd, self.path = tempfile.mkstemp(prefix=f"dg_clocks_{device_index}_", suffix=".csv")
+        os.close(fd)
         self.dev = device_index
 
     def __enter__(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             ident = self._nvsmi_id()
             self.proc = subprocess.Popen(["nvidia-smi", "-i", ident, f"--query-gpu={self.FIELDS}",
@@ -158,16 +161,27 @@ class ClockSampler:
                 self.proc.kill()
             self.f.close()
 
-    def summary(self):
+    def remove(self):
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+
+    def summary(self, t0=None, t1=None):
+        """Median SM clock and the active throttle reasons over samples in [t0, t1] (wall clock)."""
+        import datetime
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
         rows = []
         for line in open(self.path):
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 8:
+            if len(parts) < 9:
                 continue
             try:
-                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                if (t0 is not None and ts < t0) or (t1 is not None and ts > t1):
+                    continue
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
             except ValueError:
                 continue
         if not rows:
@@ -278,23 +292,30 @@ def run_gpu(args):
         dg.dg_denoise_step(p, STEP, bufs.h, W, W, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept,
                            bufs.lse, bufs.selfcond, ws, stream)
 
-    for _ in range(args.warmup):
-        step()
-    _, _, _ = dg.dg_stop_check(p, ws)
-    launches_per_step = dg.last_launch_count()
+    clk = ClockSampler(local).__enter__()          # started early: its start-up is not in the region
+    try:
+        for _ in range(args.warmup):
+            step()
+        _, _, _ = dg.dg_stop_check(p, ws)
+        launches_per_step = dg.last_launch_count()
 
-    # ---- device-timed region: K steps, inputs resident, W (1.48 GB) larger than L2
-    if world > 1:
-        tdist.barrier()
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dg.profile_enable(args.steps)
-    with ClockSampler(local) as clk:
+        # ---- device-timed region: K steps, inputs resident, W (1.48 GB) larger than L2
+        if world > 1:
+            tdist.barrier()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dg.profile_enable(args.steps)
+        t_region0 = time.time()
         ev0.record(stream)
         for _ in range(args.steps):
             step()
         ev1.record(stream)
         torch.cuda.synchronize()
+        t_region1 = time.time()
+    finally:
+        clk.__exit__(None, None, None)
+    clocks = clk.summary(t_region0, t_region1)
+    clk.remove()
     n_k1, k1_ms, _ = dg.profile_collect()
     if world > 1:
         tdist.barrier()
@@ -365,7 +386,7 @@ def run_gpu(args):
             "e2e": {"value": world * N_POS / (e2e_ms * 1e-3), "unit": "positions/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk.summary(),
+            "clocks": clocks,
             "stop_flags_after": flags,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -388,7 +409,7 @@ def run_gpu(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-rows", type=int, default=256, help="positions in the oracle's bounded CPU sample")
