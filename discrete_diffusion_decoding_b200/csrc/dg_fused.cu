@@ -676,28 +676,42 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
     const int T = a.steps_per_tile;
 
     if (tid < 32) {
-        // warp 0: merge statistics over (slot, pair) entries
-        float M = -INFINITY;
+        // warp 0: merge statistics over (slot, pair) entries.  The slots of this canvas's
+        // non-empty ranges are listed in range order, 32 ranges at a time (lane = range).
+        const int n_ct = sh_n_active;
+        const int k = ranges_per_tile(n_ct, a.n_groups);
         int ns = 0;
-        if (tid == 0) {
-            const int n_ct = sh_n_active;
-            const int k = ranges_per_tile(n_ct, a.n_groups);
-            for (int jj = 0; jj < k; ++jj) {
+        for (int j0 = 0; j0 < k; j0 += 32) {
+            const int jj = j0 + tid;
+            bool has = false;
+            int slot = 0;
+            if (jj < k) {
                 const int tb = static_cast<int>(static_cast<long long>(jj) * T / k);
                 const int te = static_cast<int>(static_cast<long long>(jj + 1) * T / k);
-                if (te <= tb) continue;
-                const long long pi = static_cast<long long>(jj) * n_ct + ct;
-                const int gg = static_cast<int>(pi % a.n_groups), round = static_cast<int>(pi / a.n_groups);
-                if (ns < kMaxSlotsPerTile) sh_slot[ns++] = gg * a.max_seg + round;
+                if (te > tb) {
+                    const long long pi = static_cast<long long>(jj) * n_ct + ct;
+                    const int gg = static_cast<int>(pi % a.n_groups), round = static_cast<int>(pi / a.n_groups);
+                    has = true;
+                    slot = gg * a.max_seg + round;
+                }
             }
-            n_slots_s = ns;
+            const uint32_t m = __ballot_sync(0xffffffffu, has);
+            const int at = ns + __popc(m & ((1u << tid) - 1u));
+            if (has && at < kMaxSlotsPerTile) sh_slot[at] = slot;
+            ns += __popc(m);
         }
+        ns = min(ns, kMaxSlotsPerTile);
+        if (tid == 0) n_slots_s = ns;
         __syncwarp();
-        ns = n_slots_s;
-        for (int s = 0; s < ns; ++s)
+        // the group reference of each slot (every pair of a piece shares it): lanes in parallel
+        float M = -INFINITY;
+        for (int s = tid; s < ns; s += 32)
             M = fmaxf(M, a.stats[(static_cast<size_t>(sh_slot[s]) * a.G) * kCanvas + crow].x);
+#pragma unroll
+        for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
         float L = 0.f, Uu = 0.f, best = -INFINITY, skey = -INFINITY;
         int bidx = 0x7fffffff, sidx = 0x7fffffff;
+#pragma unroll 4
         for (int e = tid; e < ns * a.G; e += 32) {
             const int s = e / a.G, rr = e % a.G;
             const size_t si = (static_cast<size_t>(sh_slot[s]) * a.G + rr) * kCanvas + crow;
@@ -766,6 +780,7 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
     const int col_end = min(a.d, static_cast<int>(blockIdx.y + 1) * kCombineCols);
     for (int col = static_cast<int>(blockIdx.y) * kCombineCols + tid * 4; col < col_end; col += blockDim.x * 4) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
         for (int s = 0; s < ns; ++s) {
             const float4 o =
                 *reinterpret_cast<const float4*>(a.opart + (static_cast<size_t>(sh_slot[s]) * kCanvas + crow) * a.d + col);
