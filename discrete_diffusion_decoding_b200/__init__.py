@@ -109,6 +109,12 @@ def dg_stop_check(p, ws, stream=None, want_stable=False):
     return list(flags), (list(stable) if stable is not None else None), n.value
 
 
+def dg_debug_set_error(p, ws, code, stream=None):
+    """Host-side fault injection: write `code` into the workspace's device error word."""
+    check("dg_debug_set_error", lib().dg_debug_set_error(ctypes.byref(p), ws.ptr, ws.nbytes, int(code),
+                                                         _stream(stream)))
+
+
 def dg_denoise_stats_noalloc(p, step, h, W, E, entropy, argmax, lse, selfcond, stream=None):
     """Fused pass without a caller workspace (scratch lives in the library's fixed device array)."""
     check("dg_denoise_stats_noalloc", lib().dg_denoise_stats_noalloc(

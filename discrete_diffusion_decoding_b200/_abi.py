@@ -11,7 +11,7 @@ DG_OK, DG_EINVAL, DG_ECUDA, DG_EUNSUPPORTED, DG_ETIMEOUT, DG_ENOMEM = 0, -1, -2,
 # every symbol include/dg.h declares
 EXPORTS = ("dg_params_default", "dg_temperature", "dg_workspace_size", "dg_canvas_init", "dg_denoise_step",
            "dg_stop_check", "dg_stub_hidden", "dg_status_string", "dg_last_launch_count", "dg_plan",
-           "dg_profile_enable", "dg_profile_collect", "dg_denoise_stats_noalloc")
+           "dg_profile_enable", "dg_profile_collect", "dg_denoise_stats_noalloc", "dg_debug_set_error")
 
 
 class DgParams(ctypes.Structure):
@@ -53,6 +53,8 @@ def lib():
         L.dg_denoise_step.restype = i32
         L.dg_stop_check.argtypes = [P, vp, sz, vp, vp, vp, vp]
         L.dg_stop_check.restype = i32
+        L.dg_debug_set_error.argtypes = [P, vp, sz, i32, vp]
+        L.dg_debug_set_error.restype = i32
         L.dg_stub_hidden.argtypes = [P, i32, ctypes.c_float, ctypes.c_float, vp, vp, vp, vp, vp, sz, vp]
         L.dg_stub_hidden.restype = i32
         L.dg_status_string.argtypes = [i32]

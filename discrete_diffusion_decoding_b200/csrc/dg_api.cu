@@ -457,6 +457,23 @@ dg_status dg_stop_check(const dg_params* p, void* workspace_dev, size_t workspac
     return DG_OK;
 }
 
+dg_status dg_debug_set_error(const dg_params* p, void* workspace_dev, size_t workspace_bytes, int32_t code,
+                             void* stream) {
+    const int pairs = resident_pairs();
+    if (pairs <= 0) return DG_ECUDA;
+    Plan pl;
+    dg_status st = make_plan(p, pairs, &pl);
+    if (st != DG_OK) return st;
+    if (!workspace_dev) return DG_EINVAL;
+    const Layout L = make_layout(pl);
+    if (workspace_bytes < L.total) return DG_ENOMEM;
+    // pageable source: the copy is complete when cudaMemcpyAsync returns, so `code` may live on the stack
+    if (cudaMemcpyAsync(at<int32_t>(workspace_dev, L.err), &code, sizeof(int32_t), cudaMemcpyHostToDevice,
+                        static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return DG_ECUDA;
+    return DG_OK;
+}
+
 dg_status dg_stub_hidden(const dg_params* p, int step, float gain, float noise, const uint64_t* seeds_dev,
                          const void* E_dev, const int32_t* tokens_dev, void* h_dev, void* workspace_dev,
                          size_t workspace_bytes, void* stream) {

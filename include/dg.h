@@ -159,6 +159,18 @@ dg_status dg_stop_check(const dg_params* p, void* workspace_dev, size_t workspac
                         int32_t* stable_host, int* n_stopped_host, void* stream);
 
 /*
+ * Host-side fault injection for the error path (not on the pages): writes `code`
+ * into the workspace's device error word, stream-ordered, exactly as a bounded
+ * in-kernel wait that runs out would.  The next dg_stop_check then reports
+ * DG_ETIMEOUT; dg_canvas_init clears the word.  Lets callers and tests exercise
+ * their timeout handling without making a GPU wait run out.
+ * Errors: DG_EINVAL (null workspace), DG_ENOMEM (workspace too small for p),
+ * DG_ECUDA (copy failed).
+ */
+dg_status dg_debug_set_error(const dg_params* p, void* workspace_dev, size_t workspace_bytes, int32_t code,
+                             void* stream);
+
+/*
  * Benchmark-only stand-in for the denoiser network (not on the pages):
  *   h_i = gain * (a E[tgt_i] + (1 - a) E[x_i]) + noise * n_i,   a = s / max_steps,
  * tgt_i uniform over V (Philox tag 2, step 0), n_i standard normal by Box-Muller on

@@ -306,3 +306,34 @@ def test_argument_errors(dg):
         dg.plan(bad)
     assert e.value.status == _abi.DG_EUNSUPPORTED
     assert dg.last_launch_count() == 0
+
+
+def test_forced_error_word_reported_and_cleared(dg):
+    """Host-side fault injection: a device error word (as a timed-out wait leaves it) makes the next
+    dg_stop_check return DG_ETIMEOUT; dg_canvas_init clears it; steps in between still run."""
+    from discrete_diffusion_decoding_b200 import _abi
+    V, d = 4096, 128
+    p = dg.params(1, V, d)
+    ws, bufs = dg.Workspace(p), dg.StepBuffers(p)
+    W = synth.weights(V, d).cuda()
+    seeds = torch.zeros(1, dtype=torch.int64, device="cuda")
+    dg.dg_canvas_init(p, seeds, bufs.tokens, ws)
+    bufs.h.copy_(synth.gaussian_hidden(256, d).cuda())
+    assert dg.dg_stop_check(p, ws)[2] == 0
+    dg.dg_debug_set_error(p, ws, 301)
+    dg.dg_denoise_step(p, 1, bufs.h, W, W, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept, None, None, ws)
+    with pytest.raises(_abi.DgError) as e:
+        dg.dg_stop_check(p, ws)
+    assert e.value.status == _abi.DG_ETIMEOUT
+    with pytest.raises(_abi.DgError) as e:                 # the word stays set until the canvas is re-initialised
+        dg.dg_stop_check(p, ws)
+    assert e.value.status == _abi.DG_ETIMEOUT
+    dg.dg_canvas_init(p, seeds, bufs.tokens, ws)
+    dg.dg_denoise_step(p, 1, bufs.h, W, W, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept, None, None, ws)
+    flags, _, n = dg.dg_stop_check(p, ws)
+    assert flags == [0] and n == 0
+    small = dg.Workspace(p)
+    small.nbytes = 64
+    with pytest.raises(_abi.DgError) as e:
+        dg.dg_debug_set_error(p, small, 1)
+    assert e.value.status == _abi.DG_ENOMEM
