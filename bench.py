@@ -18,6 +18,7 @@ import argparse
 import hashlib
 import json
 import math
+import re
 import os
 import statistics
 import subprocess
@@ -41,14 +42,21 @@ PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "dg_fused_kernel_single_step_v2
 CSRC = os.path.join(ROOT, "discrete_diffusion_decoding_b200", "csrc")
 
 
+def _code_only(text):
+    """C/C++ source without comments and with whitespace collapsed (comment edits do not change code)."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash():
-    """sha256 over every CUDA source and header of the library, in name order."""
+    """sha256 over the code (comments stripped) of every CUDA source and header of the library, in name order."""
     h = hashlib.sha256()
     for name in sorted(os.listdir(CSRC)):
         if name.endswith((".cu", ".cuh", ".h")):
             h.update(name.encode())
-            with open(os.path.join(CSRC, name), "rb") as f:
-                h.update(f.read())
+            with open(os.path.join(CSRC, name), encoding="utf-8") as f:
+                h.update(_code_only(f.read()).encode())
     return h.hexdigest()
 
 

@@ -25,7 +25,12 @@
 //    and then O is rescaled in TMEM.
 //  * Each CTA keeps exact per-row partial statistics of its own tiles relative
 //    to the shared reference: l = sum e, u = sum e (z - m_ref), and the best raw
-//    logit with its smallest vocabulary index.
+//    logit with its smallest vocabulary index.  The sampled-acceptance instance
+//    (dg_fused_sample_kernel) also keeps, per row, the best Gumbel-max key of the
+//    64-entry chunks' log-masses and the entry drawn inside the leading chunk.
+//  * Streamed operands carry an L2 evict-first policy; when E aliases W the
+//    first 3/10 of every W tile's hidden-column stages keep normal priority so
+//    that the self-conditioning GEMM re-reads them from L2.
 //  * Work is dealt in pieces (a range of blocks of one canvas) so that groups in
 //    the same round stream the same vocabulary rows for different canvases (rows
 //    come from DRAM once and are shared through L2); each piece ends with O and
