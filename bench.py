@@ -32,6 +32,7 @@ if ROOT not in sys.path:
 V, D, N_POS, STEP, BOUND = 262144, 2816, 256, 1, 0.1
 ACCEPT_MODE = 0            # 0: accepted positions keep the argmax; 1: a Gumbel-max sample (--accept sample)
 ACCEPT_RULE = 0            # 0: accept every position with H <= bound; 1: by groups (--rule group)
+CANVASES, UNTIED = 1, False  # per rank; other values are context measurements (--canvases, --untied)
 METRIC = "canvas positions/s per denoise step (V=262144,d=2816); % of roofline"
 WORKLOAD = ("single-step microbenchmark: 1 canvas of 256 positions, V=262144, d=2816, tied bf16 E=W ~N(0,0.02), "
             "hidden bf16 N(0,1)/sqrt(d)*8, step 1 (T=0.8), bound 0.1; outputs tokens/H/argmax/accept/self-cond fp32")
@@ -201,6 +202,20 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- CPU oracle leg
+def _set_shape(canvases, untied):
+    """--canvases C / --untied: context measurements of the batched and untied workloads (not bench lines)."""
+    global CANVASES, UNTIED, N_POS, FLOPS_PER_STEP, WE_BYTES_PER_STEP, WORKLOAD
+    CANVASES, UNTIED = int(canvases), bool(untied)
+    N_POS = 256 * CANVASES
+    FLOPS_PER_STEP = 2 * (2.0 * N_POS * V * D)
+    WE_BYTES_PER_STEP = (2.0 if UNTIED else 1.0) * 2.0 * V * D
+    if CANVASES != 1:
+        WORKLOAD = WORKLOAD.replace("1 canvas of 256 positions", f"{CANVASES} canvases of 256 positions in one launch "
+                                    "(context measurement)")
+    if UNTIED:
+        WORKLOAD = WORKLOAD.replace("tied bf16 E=W ~N(0,0.02)", "untied bf16 W, E ~N(0,0.02) (context measurement)")
+
+
 def _set_accept(mode, rule=0):
     """--accept sample / --rule group: time the sampled-acceptance kernel or the group rule."""
     global ACCEPT_MODE, ACCEPT_RULE, WORKLOAD
@@ -284,20 +299,21 @@ def run_gpu(args):
     build.build()
     import discrete_diffusion_decoding_b200 as dg
 
-    # replicas: every rank owns one canvas of its own (seed = its global canvas index)
-    c0, _ = shard_canvases(world, rank, world)
-    p = dg.params(1, V, D, accept_mode=ACCEPT_MODE, accept_rule=ACCEPT_RULE)
+    # replicas: every rank owns CANVASES canvases of its own (seed = the global canvas index)
+    c0, _ = shard_canvases(world * CANVASES, rank, world)
+    p = dg.params(CANVASES, V, D, accept_mode=ACCEPT_MODE, accept_rule=ACCEPT_RULE, tied=0 if UNTIED else 1)
     W = synth.weights(V, D, seed=1234).to(dev)
+    E = synth.weights(V, D, seed=1235).to(dev) if UNTIED else W
     h_host = synth.gaussian_hidden(N_POS, D, seed=42)
     ws = dg.Workspace(p, dev)
     bufs = dg.StepBuffers(p, dev)
-    seeds = torch.tensor([c0], dtype=torch.int64, device=dev)
+    seeds = torch.arange(c0, c0 + CANVASES, dtype=torch.int64, device=dev)
     dg.dg_canvas_init(p, seeds, bufs.tokens, ws)
     bufs.h.copy_(h_host.to(dev))
     stream = torch.cuda.current_stream()
 
     def step():
-        dg.dg_denoise_step(p, STEP, bufs.h, W, W, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept,
+        dg.dg_denoise_step(p, STEP, bufs.h, W, E, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept,
                            bufs.lse, bufs.selfcond, ws, stream)
 
     clk = ClockSampler(local).__enter__()          # started early: its start-up is not in the region
@@ -360,7 +376,7 @@ def run_gpu(args):
         for i in range(n):
             b = i % 2
             stream.wait_event(h_ready[b])
-            dg.dg_denoise_step(p, STEP, h_dev[b], W, W, seeds, bufs.tokens, bufs.entropy, bufs.argmax,
+            dg.dg_denoise_step(p, STEP, h_dev[b], W, E, seeds, bufs.tokens, bufs.entropy, bufs.argmax,
                                bufs.accept, bufs.lse, sc_dev[b], ws, stream)
             with torch.cuda.stream(stream):
                 out_H.copy_(bufs.entropy, non_blocking=True)
@@ -398,13 +414,15 @@ def run_gpu(args):
         peak_tf_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
         achieved = FLOPS_PER_STEP / (k1_max * 1e-3) / 1e12
         roof_ms = max(FLOPS_PER_STEP / (peak_tf * 1e12), WE_BYTES_PER_STEP / (float(peaks.get("hbm_gbs", 6650.0)) * 1e9)) * 1e3
-        traffic = profiled_traffic() if ACCEPT_MODE == 0 else None    # the profile is of the argmax kernel
+        # the committed DRAM capture is of the default kernel on the one-canvas tied workload
+        traffic = profiled_traffic() if (ACCEPT_MODE == 0 and CANVASES == 1 and not UNTIED) else None
         value = world * N_POS / (ms_per_step * 1e-3)
         line = {
             "metric": METRIC, "value": value, "unit": "positions/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "n_canvas": world, "positions": world * N_POS, "vocab": V, "hidden": D,
+            "config": {"workload": WORKLOAD, "n_canvas": world * CANVASES, "positions": world * N_POS, "vocab": V,
+                       "hidden": D,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2 (W/E 1.48 GB streamed per step)",
                        "group": dg.plan(p)["group"], "n_groups": dg.plan(p)["n_groups"]},
@@ -422,7 +440,7 @@ def run_gpu(args):
             "clocks": clocks,
             "stop_flags_after": flags,
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and CANVASES == 1 and not UNTIED:
             # bounded sample of the same workload through the float64 oracle on the host cores
             from oracle import stage
             W64 = stage.bf16_to_f64(synth.bf16_bits(W.cpu()))
@@ -451,12 +469,16 @@ def main(argv=None):
                     help="token kept at accepted positions (sample: Gumbel-max draw from softmax(z/T))")
     ap.add_argument("--rule", choices=["position", "group"], default="position",
                     help="accepted positions: H <= bound each, or the canvas's entropy-ordered group within the bound")
+    ap.add_argument("--canvases", type=int, default=1,
+                    help="canvases per rank in one launch; values other than 1 are context measurements, not bench lines")
+    ap.add_argument("--untied", action="store_true", help="separate W and E (context measurement, not a bench line)")
     ap.add_argument("--vocab", type=int, default=262144,
                     help="vocabulary size; smaller values are for profiler captures only, not bench lines")
     args = ap.parse_args(argv)
     if args.vocab != V:
         _set_vocab(args.vocab)
     _set_accept(1 if args.accept == "sample" else 0, 1 if args.rule == "group" else 0)
+    _set_shape(args.canvases, args.untied)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
