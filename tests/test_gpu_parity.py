@@ -337,3 +337,52 @@ def test_forced_error_word_reported_and_cleared(dg):
     with pytest.raises(_abi.DgError) as e:
         dg.dg_debug_set_error(p, small, 1)
     assert e.value.status == _abi.DG_ENOMEM
+
+
+def test_all_canvases_stopped_step_is_a_no_op(dg):
+    """Empty work: once every canvas has stopped, a further step (and the stub) leaves every output as it was."""
+    V, d, C, S = 4096, 128, 2, 16
+    W = synth.weights(V, d)
+    Wd = W.cuda()
+    p = dg.params(C, V, d, max_steps=S)
+    ws, bufs = dg.Workspace(p), dg.StepBuffers(p)
+    seeds = torch.tensor(np.asarray(synth.canvas_seeds(C, base=70), np.uint64).view(np.int64), device="cuda")
+    dg.dg_canvas_init(p, seeds, bufs.tokens, ws)
+    s_stop = None
+    for s in range(1, S + 1):
+        dg.dg_stub_hidden(p, s, 300.0, 0.1, seeds, Wd, bufs.tokens, bufs.h, ws)
+        dg.dg_denoise_step(p, s, bufs.h, Wd, Wd, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept,
+                           bufs.lse, bufs.selfcond, ws)
+        _, _, n = dg.dg_stop_check(p, ws)
+        if n == C:
+            s_stop = s
+            break
+    assert s_stop is not None and s_stop < S, "both canvases should stop early at gain 300"
+    before = {k: getattr(bufs, k).clone() for k in ("h", "tokens", "entropy", "argmax", "accept", "lse", "selfcond")}
+    dg.dg_stub_hidden(p, s_stop + 1, 300.0, 0.1, seeds, Wd, bufs.tokens, bufs.h, ws)
+    dg.dg_denoise_step(p, s_stop + 1, bufs.h, Wd, Wd, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept,
+                       bufs.lse, bufs.selfcond, ws)
+    flags, _, n = dg.dg_stop_check(p, ws)
+    assert flags == [1] * C and n == C
+    for k, v in before.items():
+        assert torch.equal(getattr(bufs, k), v), f"{k} changed in a step with no active canvas"
+
+
+def test_maximum_canvases_per_launch(dg):
+    """256 canvases (N = 65536) in one launch: sampled rows of many canvases against the oracle; 257 is refused."""
+    from discrete_diffusion_decoding_b200 import _abi
+    V, d, C = 4096, 128, 256
+    W = synth.weights(V, d)
+    h, _ = synth.spiked_hidden(W, C * 256, seed=90, gain_lo=0.5, gain_hi=20.0)
+    p = dg.params(C, V, d)
+    seeds = synth.canvas_seeds(C, base=500)
+    Wd = W.cuda()
+    g = gc.gpu_step(dg, p, 2, h, Wd, Wd, seeds)
+    rng = np.random.default_rng(12)
+    rows = np.unique(np.concatenate([[0, 255, 256, C * 256 - 1], rng.choice(C * 256, 60, replace=False)]))
+    o = gc.oracle_rows(gc.bits(h), gc.bits(W), gc.bits(W), dg.temperature(p, 2), p.eb_bound, seeds, 2, rows, V)
+    gc.compare(g, o, rows, p.eb_bound, tag="256 canvases")
+    assert np.all(g["stable"] == 0) and np.all(g["stop"] == 0)      # step 2 of a fresh run: nothing stable yet
+    with pytest.raises(_abi.DgError) as e:
+        dg.workspace_size(dg.params(C + 1, V, d))
+    assert e.value.status == _abi.DG_EINVAL
