@@ -130,3 +130,44 @@ def test_group_lockstep_decode_small(dg):
         if all(stopped):
             break
     assert checked >= 6 and accepted > 0
+
+
+def test_sampled_group_lockstep_decode_small(dg):
+    """Both options at once over a stub-driven decode: the group rule picks the accepted set, accepted
+    positions keep the two-level sample; every step against the oracle (lock-step on the GPU's h)."""
+    V, d, C, S, gain = 4096, 128, 2, 12, 300.0
+    W = synth.weights(V, d)
+    Wb = gc.bits(W)
+    p = dg.params(C, V, d, max_steps=S, eb_bound=10.0, accept_rule=1, accept_mode=1)   # wide: spread rows kept
+    ws, bufs = dg.Workspace(p), dg.StepBuffers(p)
+    seeds = synth.canvas_seeds(C, base=60)
+    seeds_t = torch.tensor(np.asarray(seeds, np.uint64).view(np.int64), device="cuda")
+    Wd = W.cuda()
+    dg.dg_canvas_init(p, seeds_t, bufs.tokens, ws)
+    checked = differ = 0
+    stopped = [False] * C
+    for s in range(1, S + 1):
+        dg.dg_stub_hidden(p, s, gain, 0.1, seeds_t, Wd, bufs.tokens, bufs.h, ws)
+        dg.dg_denoise_step(p, s, bufs.h, Wd, Wd, seeds_t, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept,
+                           bufs.lse, bufs.selfcond, ws)
+        flags, _, _ = dg.dg_stop_check(p, ws)
+        g = {"H": bufs.entropy.cpu().numpy().astype(np.float64), "argmax": bufs.argmax.cpu().numpy(),
+             "tokens": bufs.tokens.cpu().numpy().astype(np.int64), "accept": bufs.accept.cpu().numpy()}
+        hb = gc.bits(bufs.h)
+        T = dg.temperature(p, s)
+        for c in range(C):
+            if stopped[c]:
+                continue
+            rows = np.arange(c * 256, (c + 1) * 256)
+            o = stage.step_rows(hb[rows], Wb, Wb, T, p.eb_bound, int(seeds[c]), s, c, np.arange(256), V,
+                                want_selfcond=False, accept_mode=1)
+            ok_arg = o["top2gap"] >= gc.EXCL
+            assert np.array_equal(g["argmax"][rows][ok_arg], o["argmax"][ok_arg]), f"argmax s={s} c={c}"
+            kept_ok = (o["keygap"] >= gc.EXCL) & (o["cdf_margin"] >= 1e-4)
+            if _check_canvas(g, c, o["H"], o["sample"], kept_ok, p.eb_bound, int(seeds[c]), s, V, f"s={s} c={c}"):
+                checked += 1
+                differ += int(np.sum((g["accept"][rows] == 1) & (o["sample"] != o["argmax"])))
+            stopped[c] = bool(flags[c])
+        if all(stopped):
+            break
+    assert checked >= 6 and differ >= 3
