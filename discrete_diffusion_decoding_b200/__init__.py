@@ -15,7 +15,7 @@ from ._abi import DgError, DgParams, check, lib
 
 __all__ = ["DgError", "DgParams", "params", "workspace_size", "plan", "temperature", "dg_canvas_init",
            "dg_denoise_step", "dg_stop_check", "dg_stub_hidden", "last_launch_count", "profile_enable",
-           "profile_collect", "dg_denoise_stats_noalloc", "Workspace", "StepBuffers",
+           "profile_collect", "dg_denoise_stats_noalloc", "dg_debug_set_error", "Workspace", "StepBuffers",
            "decode_batch", "decode_block_ar"]
 
 
