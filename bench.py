@@ -413,7 +413,11 @@ def run_gpu(args):
         peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
         peak_tf_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
         achieved = FLOPS_PER_STEP / (k1_max * 1e-3) / 1e12
-        roof_ms = max(FLOPS_PER_STEP / (peak_tf * 1e12), WE_BYTES_PER_STEP / (float(peaks.get("hbm_gbs", 6650.0)) * 1e9)) * 1e3
+        # the fused kernel is timed inside a seconds-long loop under the power cap, the regime of the
+        # sustained (back-to-back) GEMM measurement, so that is the peak; the burst one is reported beside it
+        hbm = float(peaks.get("hbm_gbs", 6650.0)) * 1e9
+        roof_ms = max(FLOPS_PER_STEP / (peak_tf_sus * 1e12), WE_BYTES_PER_STEP / hbm) * 1e3
+        roof_ms_burst = max(FLOPS_PER_STEP / (peak_tf * 1e12), WE_BYTES_PER_STEP / hbm) * 1e3
         # the committed DRAM capture is of the default kernel on the one-canvas tied workload
         traffic = profiled_traffic() if (ACCEPT_MODE == 0 and CANVASES == 1 and not UNTIED) else None
         value = world * N_POS / (ms_per_step * 1e-3)
@@ -427,13 +431,16 @@ def run_gpu(args):
                        "l2": "inputs larger than L2 (W/E 1.48 GB streamed per step)",
                        "group": dg.plan(p)["group"], "n_groups": dg.plan(p)["n_groups"]},
             "steps_per_s": 1e3 / ms_per_step,
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
-                         "frac": achieved / peak_tf, "traffic": traffic,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf_sus, "unit": "TFLOP/s",
+                         "frac": achieved / peak_tf_sus, "traffic": traffic,
                          "kernel": "dg_fused_sample_kernel" if ACCEPT_MODE else "dg_fused_kernel",
                          "kernel_ms": k1_max, "launches_timed": n_k1,
-                         "flops_per_launch": FLOPS_PER_STEP, "peak_source": f"{peaks_src} bf16 burst",
-                         "frac_of_sustained": achieved / peak_tf_sus,
-                         "step_frac": roof_ms / ms_per_step, "roofline_step_ms": roof_ms},
+                         "flops_per_launch": FLOPS_PER_STEP,
+                         "peak_source": f"{peaks_src} bf16 sustained (back-to-back GEMM loop under the power cap, "
+                                        "the regime the kernel is timed in)",
+                         "burst_peak": peak_tf, "frac_of_burst": achieved / peak_tf,
+                         "step_frac": roof_ms / ms_per_step, "roofline_step_ms": roof_ms,
+                         "roofline_step_ms_at_burst": roof_ms_burst},
             "e2e": {"value": world * N_POS / (e2e_ms * 1e-3), "unit": "positions/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
