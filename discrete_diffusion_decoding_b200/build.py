@@ -29,20 +29,28 @@ def _stale():
 
 
 def build(force=False, verbose=False):
-    """Compile libdg.so if missing or older than its sources; returns the library path."""
+    """Compile libdg.so if missing or older than its sources; returns the library path.
+
+    Safe when several processes (one per GPU) build at once: each compiles into its own
+    temporary file and renames it over the library atomically; a process that has already
+    loaded the library keeps its mapping.
+    """
     if not force and not _stale():
         return LIB
+    tmp = f"{LIB}.{os.getpid()}.tmp"
     cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
-           "-Xcompiler", "-fPIC", "-shared", "-o", LIB + ".tmp"] + [os.path.join(CSRC, s) for s in SOURCES]
+           "-Xcompiler", "-fPIC", "-shared", "-o", tmp] + [os.path.join(CSRC, s) for s in SOURCES]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
+        if os.path.exists(tmp):
+            os.remove(tmp)
         raise RuntimeError("nvcc failed building libdg.so")
     if verbose:
         sys.stderr.write(res.stderr)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(tmp, LIB)
     return LIB
 
 
