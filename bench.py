@@ -291,20 +291,25 @@ def run_gpu(args):
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        tdist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
 
     import synth
     from discrete_diffusion_decoding_b200 import build
     build.build()
     import discrete_diffusion_decoding_b200 as dg
 
-    # replicas: every rank owns CANVASES canvases of its own (seed = the global canvas index)
-    c0, _ = shard_canvases(world * CANVASES, rank, world)
-    p = dg.params(CANVASES, V, D, accept_mode=ACCEPT_MODE, accept_rule=ACCEPT_RULE, tied=0 if UNTIED else 1)
+    # inputs first, each rank with its share of the host's cores, so that the ranks reach the
+    # process group (and its short timeout) together
+    if world > 1:
+        torch.set_num_threads(max(1, (os.cpu_count() or 1) // world))
     W = synth.weights(V, D, seed=1234).to(dev)
     E = synth.weights(V, D, seed=1235).to(dev) if UNTIED else W
     h_host = synth.gaussian_hidden(N_POS, D, seed=42)
+    if world > 1:
+        tdist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+
+    # replicas: every rank owns CANVASES canvases of its own (seed = the global canvas index)
+    c0, _ = shard_canvases(world * CANVASES, rank, world)
+    p = dg.params(CANVASES, V, D, accept_mode=ACCEPT_MODE, accept_rule=ACCEPT_RULE, tied=0 if UNTIED else 1)
     ws = dg.Workspace(p, dev)
     bufs = dg.StepBuffers(p, dev)
     seeds = torch.arange(c0, c0 + CANVASES, dtype=torch.int64, device=dev)
