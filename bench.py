@@ -12,6 +12,8 @@ stop reduction.  Inputs are larger than L2 (W streams 1.48 GB per step).
 Prints one JSON line (rank 0).  With --gpus N > 1 (under torchrun) every rank
 runs an independent replica (canvases shard across GPUs with no data-path
 collective); the value is all ranks' positions over the slowest rank's time.
+With --split vocab the ranks instead share one canvas and split the head by
+vocabulary rows (an all-gather of the shards' partials each step).
 """
 
 import argparse
@@ -21,7 +23,6 @@ import math
 import re
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -126,79 +127,83 @@ def profiled_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms; summary() keeps the samples
-    whose timestamps fall inside the timed region (the sampler is started before the warm-up
-    so that its start-up does not eat into the region)."""
+    """SM clock, power and clock-event (throttle) reasons sampled through NVML every 2 ms on a
+    background thread; summary() keeps the samples whose timestamps fall inside the timed region
+    (the sampler is started before the warm-up so that its start-up does not eat into the region).
+    A 20-step region of ~13 ms still gets several samples."""
 
-    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
 
-    def __init__(self, device_index):
-        import tempfile
-        self.proc = None
-        fd, self.path = tempfile.mkstemp(prefix=f"dg_clocks_{device_index}_", suffix=".csv")
-        os.close(fd)
-        self.dev = device_index
+    def __init__(self, device_index, period_s=0.002):
+        self.dev, self.period, self.rows, self.err = device_index, period_s, [], None
+        self._stop = None
+        self._thread = None
 
-    def __enter__(self):
-        try:
-            self.f = open(self.path, "w")
-            ident = self._nvsmi_id()
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", ident, f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=self.f, stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
-        return self
-
-    def _nvsmi_id(self):
+    def _handle(self):
+        import pynvml
         import torch
+        pynvml.nvmlInit()
         try:
             pr = torch.cuda.get_device_properties(self.dev)
-            return f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
         except Exception:
-            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-            return vis.split(",")[self.dev] if vis else str(self.dev)
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+
+    def __enter__(self):
+        import threading
+        try:
+            nv, h = self._handle()
+        except Exception as e:           # no NVML: the line says so
+            self.err = f"nvml unavailable: {e}"
+            return self
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    self.rows.append((time.time(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                      nv.nvmlDeviceGetPowerUsage(h) / 1000.0, int(get_reasons(h))))
+                except Exception as e:
+                    self.err = str(e)
+                    return
+                time.sleep(self.period)
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+        return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.f.close()
-
-    def remove(self):
-        try:
-            os.remove(self.path)
-        except OSError:
-            pass
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
 
     def summary(self, t0=None, t1=None):
-        """Median SM clock and the active throttle reasons over samples in [t0, t1] (wall clock)."""
-        import datetime
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
-        rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
-                if (t0 is not None and ts < t0) or (t1 is not None and ts > t1):
-                    continue
-                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-            except ValueError:
-                continue
+        """Median SM clock, max clock, median power and the reasons active in any sample of [t0, t1]."""
+        if self.err and not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err], "samples": 0}
+        rows = [r for r in self.rows if (t0 is None or r[0] >= t0) and (t1 is None or r[0] <= t1)]
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, st in rows for i, v in enumerate(st) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({name for _, _, _, bits in rows for name, bit in self.REASONS if bits & bit})
+        return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": self.max_mhz,
+                "power_w": round(statistics.median(r[2] for r in rows), 1), "reasons": reasons,
+                "samples": len(rows), "source": "nvml, 2 ms"}
+
+
+def choose_peak(peaks, region_s, clocks):
+    """The bf16 peak that matches the regime the fused kernel was timed in: the sustained figure
+    (a seconds-long GEMM loop under the power cap) when the timed region lasted at least a second
+    and the power cap was active in it; the burst figure otherwise.  Returns (peak, name)."""
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    capped = "sw_power_cap" in (clocks.get("reasons") or [])
+    if region_s >= 1.0 and capped:
+        return sustained, "sustained"
+    return burst, "burst"
 
 
 # ----------------------------------------------------------------------------- CPU oracle leg
@@ -249,7 +254,12 @@ def oracle_sample_rate(W64, h_bits, n_rows, T):
 
 
 def run_reference(args):
-    """--impl reference: the float64 CPU oracle as it stands, timed on the host cores."""
+    """--impl reference: the float64 CPU oracle as it stands, timed on the host cores.
+
+    Every timed step is a whole 256-position step when K of them fit in about two minutes
+    (the driver's short runs); otherwise each step is a bounded sample of positions and the
+    line says so (ms_per_step is then scaled to a whole step and marked as such).
+    """
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
@@ -260,31 +270,87 @@ def run_reference(args):
     W64, hb = stage.bf16_to_f64(synth.bf16_bits(W)), synth.bf16_bits(h)
     del W
     T = stage.temperature(STEP, 48)
-    # bounded sample per step: size it from one probe so the whole run stays within about two minutes
-    _, probe_dt, _ = oracle_sample_rate(W64, hb, 1, T)
-    n_rows = int(max(1, min(N_POS, 120.0 / max(1, args.steps + args.warmup) / probe_dt)))
+    _, probe_dt, _ = oracle_sample_rate(W64, hb, 8, T)
+    full_est = probe_dt * N_POS / 8
+    n_rows = N_POS if args.steps * full_est <= 120.0 else int(max(1, min(N_POS, 120.0 / args.steps / probe_dt * 8)))
     for _ in range(args.warmup):
-        oracle_sample_rate(W64, hb, 1, T)
+        oracle_sample_rate(W64, hb, 1, T)          # untimed warm-up: one position per step
     times, threads = [], 1
     for _ in range(args.steps):
-        rate, dt, threads = oracle_sample_rate(W64, hb, n_rows, T)
+        _, dt, threads = oracle_sample_rate(W64, hb, n_rows, T)
         times.append(dt)
-    ms = statistics.mean(times) * 1e3 * (N_POS / n_rows)     # scaled to a full 256-position step
+    measured_ms = statistics.mean(times) * 1e3
+    ms = measured_ms * (N_POS / n_rows)
     value = N_POS / (ms * 1e-3)
+    whole = n_rows == N_POS
+    sample = ("every timed step is a whole 256-position step" if whole else
+              f"{n_rows} of 256 positions per timed step ({measured_ms:.0f} ms), scaled to a whole step")
     line = {"metric": METRIC, "value": value, "unit": "positions/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms,
+            "ms_per_step_kind": "measured whole steps" if whole else f"scaled from {n_rows} of 256 positions",
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": WORKLOAD, "n_canvas": 1, "positions": N_POS, "vocab": V, "hidden": D},
             "cpu_baseline": {"value": value, "unit": "positions/s", "cores": threads, "kind": "oracle",
-                             "sample": f"{n_rows} of 256 positions per step, scaled to a full step"},
+                             "sample": sample},
             "e2e": {"value": value, "unit": "positions/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
+def run_cpu_configs(args):
+    """--cpu-configs: the float64 oracle on the host cores for the other workloads (context lines,
+    one per workload): the small decode timed in full (all 16 steps of its schedule, its stub
+    included), and one step of the block decode, the 16-canvas batch and the 4-canvas untied
+    adversarial batch at their sizes, multiplied by the steps of a 48-step schedule and marked
+    "extrapolated"."""
+    import numpy as np
+    import synth
+    from oracle import decode, stage
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        threads = os.cpu_count() or 1
+
+    def emit(workload, positions, seconds, kind, extra):
+        rate = positions / seconds
+        print(json.dumps({"metric": METRIC, "impl": "reference", "kind": "context (not a bench line)",
+                          "config": {"workload": workload},
+                          "cpu_baseline": {"value": rate, "unit": "positions/s", "cores": threads,
+                                           "kind": "oracle", "sample": kind, **extra}}), flush=True)
+
+    # small decode: V=4096, d=128, 1 canvas, literal stub, 16 steps, timed in full
+    Ws = synth.bf16_bits(synth.weights(4096, 128))
+    seeds = synth.canvas_seeds(1)
+    t0 = time.perf_counter()
+    r = decode.decode_batch(Ws, Ws, seeds, decode.stub_hidden_fn(Ws, seeds, 16, 1.0, 0.1), 4096, max_steps=16)
+    dt = time.perf_counter() - t0
+    emit("small decode: 1 canvas, V=4096, d=128, stub gain 1, 16-step schedule", 256 * int(r["stop_step"][0]), dt,
+         f"timed in full: {int(r['stop_step'][0])} steps in {dt:.2f} s", {"steps": int(r["stop_step"][0])})
+    # full-size workloads: one step each, extrapolated to the 48-step schedule
+    W = synth.weights(V, D, seed=1234)
+    W64 = stage.bf16_to_f64(synth.bf16_bits(W))
+    T = stage.temperature(1, 48)
+    for name, C, untied in (("block decode: 8 canvases of 256 one after another", 1, False),
+                            ("16 canvases in one launch (N=4096)", 16, False),
+                            ("4 canvases (N=1024), untied W and E", 4, True)):
+        E64 = stage.bf16_to_f64(synth.bf16_bits(synth.weights(V, D, seed=1235))) if untied else W64
+        h = synth.bf16_bits(synth.gaussian_hidden(C * 256, D, seed=42))
+        t0 = time.perf_counter()
+        for c in range(C):
+            stage.step_rows(h[c * 256:(c + 1) * 256], W64, E64, T, BOUND, c, 1, c, np.arange(256), V)
+        dt = time.perf_counter() - t0
+        total_steps = 48 * (8 if C == 1 else 1)
+        emit(name + ", V=262144, d=2816, 48-step schedule", C * 256, dt,
+             f"extrapolated: one step of {C * 256} positions took {dt:.1f} s; a 48-step decode of the "
+             f"workload would take about {dt * total_steps / 60:.0f} min", {"one_step_s": dt})
+        del E64
+    return 0
+
+
 # ----------------------------------------------------------------------------- GPU leg
 def run_gpu(args):
-    import numpy as np
     import torch
     import torch.distributed as tdist
 
@@ -296,37 +362,58 @@ def run_gpu(args):
     from discrete_diffusion_decoding_b200 import build
     build.build()
     import discrete_diffusion_decoding_b200 as dg
+    from discrete_diffusion_decoding_b200 import vocab_parallel as vp
 
+    split = args.split == "vocab" and world > 1
     # inputs first, each rank with its share of the host's cores, so that the ranks reach the
     # process group (and its short timeout) together
     if world > 1:
         torch.set_num_threads(max(1, (os.cpu_count() or 1) // world))
-    W = synth.weights(V, D, seed=1234).to(dev)
-    E = synth.weights(V, D, seed=1235).to(dev) if UNTIED else W
+    W_host = synth.weights(V, D, seed=1234)
+    if split:
+        v0, v1 = vp.shard_bounds(V, world, rank)
+        W = W_host[v0:v1].contiguous().to(dev)
+        E = synth.weights(V, D, seed=1235)[v0:v1].contiguous().to(dev) if UNTIED else W
+    else:
+        v0, v1 = 0, V
+        W = W_host.to(dev)
+        E = synth.weights(V, D, seed=1235).to(dev) if UNTIED else W
+    del W_host
     h_host = synth.gaussian_hidden(N_POS, D, seed=42)
     if world > 1:
         tdist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
 
-    # replicas: every rank owns CANVASES canvases of its own (seed = the global canvas index)
-    c0, _ = shard_canvases(world * CANVASES, rank, world)
+    # replicas: every rank owns CANVASES canvases of its own (seed = the global canvas index);
+    # vocabulary split: every rank works on the same canvases over its rows of the head
+    c0 = 0 if split else shard_canvases(world * CANVASES, rank, world)[0]
     p = dg.params(CANVASES, V, D, accept_mode=ACCEPT_MODE, accept_rule=ACCEPT_RULE, tied=0 if UNTIED else 1)
-    ws = dg.Workspace(p, dev)
     bufs = dg.StepBuffers(p, dev)
     seeds = torch.arange(c0, c0 + CANVASES, dtype=torch.int64, device=dev)
-    dg.dg_canvas_init(p, seeds, bufs.tokens, ws)
-    bufs.h.copy_(h_host.to(dev))
     stream = torch.cuda.current_stream()
+    if split:
+        stepper = vp.SplitStep(p, W, E, v0, v1)
+        ws = stepper.ws
+        stepper.init(seeds, bufs.tokens)
+    else:
+        ws = dg.Workspace(p, dev)
+        dg.dg_canvas_init(p, seeds, bufs.tokens, ws)
+    bufs.h.copy_(h_host.to(dev))
 
-    def step():
-        dg.dg_denoise_step(p, STEP, bufs.h, W, E, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept,
-                           bufs.lse, bufs.selfcond, ws, stream)
+    def step(h=None, sc=None):
+        h = bufs.h if h is None else h
+        if split:
+            stepper(STEP, h, seeds, bufs, stream, selfcond=sc)
+        else:
+            dg.dg_denoise_step(p, STEP, h, W, E, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept,
+                               bufs.lse, bufs.selfcond if sc is None else sc, ws, stream)
 
     clk = ClockSampler(local).__enter__()          # started early: its start-up is not in the region
     try:
         for _ in range(args.warmup):
             step()
         _, _, _ = dg.dg_stop_check(p, ws)
-        launches_per_step = dg.last_launch_count()
+        step()
+        launches_per_step = 4 if split else dg.last_launch_count()   # split: partial (2) + merge (2)
 
         # ---- device-timed region: K steps, inputs resident, W (1.48 GB) larger than L2
         if world > 1:
@@ -344,7 +431,6 @@ def run_gpu(args):
     finally:
         clk.__exit__(None, None, None)
     clocks = clk.summary(t_region0, t_region1)
-    clk.remove()
     n_k1, k1_ms, _ = dg.profile_collect()
     if world > 1:
         tdist.barrier()
@@ -365,7 +451,7 @@ def run_gpu(args):
     out_am = torch.empty(N_POS, dtype=torch.int32).pin_memory()
     out_acc = torch.empty(N_POS, dtype=torch.uint8).pin_memory()
     out_sc = [torch.empty((N_POS, D), dtype=torch.float32).pin_memory() for _ in range(2)]
-    e2e_steps = args.steps            # as long as the device-timed loop: the same power-capped clock regime
+    e2e_steps = args.steps            # as long as the device-timed loop: the same clock regime
     copy_stream = torch.cuda.Stream(device=dev)
     h_dev = [bufs.h, torch.empty_like(bufs.h)]
     sc_dev = [bufs.selfcond, torch.empty_like(bufs.selfcond)]
@@ -381,8 +467,7 @@ def run_gpu(args):
         for i in range(n):
             b = i % 2
             stream.wait_event(h_ready[b])
-            dg.dg_denoise_step(p, STEP, h_dev[b], W, E, seeds, bufs.tokens, bufs.entropy, bufs.argmax,
-                               bufs.accept, bufs.lse, sc_dev[b], ws, stream)
+            step(h_dev[b], sc_dev[b])
             with torch.cuda.stream(stream):
                 out_H.copy_(bufs.entropy, non_blocking=True)
                 out_tok.copy_(bufs.tokens, non_blocking=True)
@@ -415,43 +500,52 @@ def run_gpu(args):
     line = None
     if rank == 0:
         peaks, peaks_src = load_peaks()
-        peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-        peak_tf_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-        achieved = FLOPS_PER_STEP / (k1_max * 1e-3) / 1e12
-        # the fused kernel is timed inside a seconds-long loop under the power cap, the regime of the
-        # sustained (back-to-back) GEMM measurement, so that is the peak; the burst one is reported beside it
-        hbm = float(peaks.get("hbm_gbs", 6650.0)) * 1e9
-        roof_ms = max(FLOPS_PER_STEP / (peak_tf_sus * 1e12), WE_BYTES_PER_STEP / hbm) * 1e3
-        roof_ms_burst = max(FLOPS_PER_STEP / (peak_tf * 1e12), WE_BYTES_PER_STEP / hbm) * 1e3
+        peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        region_s = elapsed_max * 1e-3
+        peak_tf, regime = choose_peak(peaks, region_s, clocks)
+        rows_per_rank = v1 - v0
+        flops_launch = 2 * (2.0 * N_POS * rows_per_rank * D)
+        achieved = flops_launch / (k1_max * 1e-3) / 1e12
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])) * 1e9
+        bytes_launch = (2.0 if UNTIED else 1.0) * 2.0 * rows_per_rank * D
+        roof_ms = max(flops_launch / (peak_tf * 1e12), bytes_launch / hbm) * 1e3
         # the committed DRAM capture is of the default kernel on the one-canvas tied workload
-        traffic = profiled_traffic() if (ACCEPT_MODE == 0 and CANVASES == 1 and not UNTIED) else None
-        value = world * N_POS / (ms_per_step * 1e-3)
+        traffic = profiled_traffic() if (ACCEPT_MODE == 0 and CANVASES == 1 and not UNTIED and not split) else None
+        positions = (1 if split else world) * N_POS
+        value = positions / (ms_per_step * 1e-3)
         line = {
             "metric": METRIC, "value": value, "unit": "positions/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "strong" if split else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "n_canvas": world * CANVASES, "positions": world * N_POS, "vocab": V,
-                       "hidden": D,
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "config": {"workload": WORKLOAD, "n_canvas": (1 if split else world) * CANVASES, "positions": positions,
+                       "vocab": V, "hidden": D,
+                       "parallelism": (f"vocabulary split x{world} (all-gather of shard partials)" if split else
+                                       f"replicas x{world}" if world > 1 else "single GPU"),
                        "l2": "inputs larger than L2 (W/E 1.48 GB streamed per step)",
                        "group": dg.plan(p)["group"], "n_groups": dg.plan(p)["n_groups"]},
             "steps_per_s": 1e3 / ms_per_step,
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf_sus, "unit": "TFLOP/s",
-                         "frac": achieved / peak_tf_sus, "traffic": traffic,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": achieved / peak_tf, "traffic": traffic,
                          "kernel": "dg_fused_sample_kernel" if ACCEPT_MODE else "dg_fused_kernel",
-                         "kernel_ms": k1_max, "launches_timed": n_k1,
-                         "flops_per_launch": FLOPS_PER_STEP,
-                         "peak_source": f"{peaks_src} bf16 sustained (back-to-back GEMM loop under the power cap, "
-                                        "the regime the kernel is timed in)",
-                         "burst_peak": peak_tf, "frac_of_burst": achieved / peak_tf,
-                         "step_frac": roof_ms / ms_per_step, "roofline_step_ms": roof_ms,
-                         "roofline_step_ms_at_burst": roof_ms_burst},
-            "e2e": {"value": world * N_POS / (e2e_ms * 1e-3), "unit": "positions/s", "h2d_bytes_per_step": h2d,
+                         "kernel_ms": k1_max, "launches_timed": n_k1, "flops_per_launch": flops_launch,
+                         "peak_regime": regime,
+                         "peak_source": (f"{peaks_src} bf16 {regime}: " +
+                                         ("a seconds-long GEMM loop under the power cap; the timed region lasted "
+                                          f"{region_s:.2f} s with sw_power_cap active" if regime == "sustained" else
+                                          f"a short GEMM burst; the timed region lasted {region_s:.3f} s")),
+                         "frac_of_burst": achieved / peak_burst, "frac_of_sustained": achieved / peak_sus,
+                         "burst_peak": peak_burst, "sustained_peak": peak_sus,
+                         "step_frac": roof_ms / ms_per_step, "roofline_step_ms": roof_ms},
+            "e2e": {"value": positions / (e2e_ms * 1e-3), "unit": "positions/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
             "stop_flags_after": flags,
         }
+        if split:
+            line["multi_gpu_note"] = "vocabulary split: NCCL all-gather of each rank's partial, merge on every rank"
         if world == 1 and not args.no_cpu_baseline and CANVASES == 1 and not UNTIED:
             # bounded sample of the same workload through the float64 oracle on the host cores
             from oracle import stage
@@ -477,6 +571,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-rows", type=int, default=256, help="positions in the oracle's bounded CPU sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-configs", action="store_true",
+                    help="time the float64 oracle on the other workloads (context lines) and exit")
     ap.add_argument("--accept", choices=["argmax", "sample"], default="argmax",
                     help="token kept at accepted positions (sample: Gumbel-max draw from softmax(z/T))")
     ap.add_argument("--rule", choices=["position", "group"], default="position",
@@ -484,6 +580,9 @@ def main(argv=None):
     ap.add_argument("--canvases", type=int, default=1,
                     help="canvases per rank in one launch; values other than 1 are context measurements, not bench lines")
     ap.add_argument("--untied", action="store_true", help="separate W and E (context measurement, not a bench line)")
+    ap.add_argument("--split", choices=["replicas", "vocab"], default="replicas",
+                    help="with --gpus N > 1: independent replicas (weak scaling, default) or one head split by "
+                         "vocabulary rows over the ranks (strong scaling)")
     ap.add_argument("--vocab", type=int, default=262144,
                     help="vocabulary size; smaller values are for profiler captures only, not bench lines")
     args = ap.parse_args(argv)
@@ -493,6 +592,8 @@ def main(argv=None):
     _set_shape(args.canvases, args.untied)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.cpu_configs:
+        return run_cpu_configs(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)

@@ -16,7 +16,7 @@ from ._abi import DgError, DgParams, check, lib
 __all__ = ["DgError", "DgParams", "params", "workspace_size", "plan", "temperature", "dg_canvas_init",
            "dg_denoise_step", "dg_stop_check", "dg_stub_hidden", "last_launch_count", "profile_enable",
            "profile_collect", "dg_denoise_stats_noalloc", "dg_debug_set_error", "Workspace", "StepBuffers",
-           "decode_batch", "decode_block_ar"]
+           "decode_batch", "decode_block_ar", "dg_partial_bytes", "dg_denoise_partial", "dg_denoise_merge"]
 
 
 def params(n_canvas, vocab, hidden, **overrides):
@@ -122,6 +122,29 @@ def dg_denoise_stats_noalloc(p, step, h, W, E, entropy, argmax, lse, selfcond, s
         _ptr(selfcond), _stream(stream)))
 
 
+def dg_partial_bytes(p):
+    """Bytes of one vocabulary shard's partial (statistics + self-conditioning numerator)."""
+    n = lib().dg_partial_bytes(ctypes.byref(p))
+    if n == 0:
+        raise DgError("dg_partial_bytes", _abi.DG_EINVAL, "invalid params")
+    return n
+
+
+def dg_denoise_partial(p, step, v_begin, v_count, h, W_shard, E_shard, seeds, partial, ws, stream=None):
+    """Fused pass over vocabulary rows [v_begin, v_begin + v_count) into `partial` (uint8 device buffer)."""
+    check("dg_denoise_partial", lib().dg_denoise_partial(
+        ctypes.byref(p), int(step), int(v_begin), int(v_count), _ptr(h), _ptr(W_shard), _ptr(E_shard), _ptr(seeds),
+        _ptr(partial), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def dg_denoise_merge(p, step, n_parts, partials, seeds, tokens, entropy, argmax, accept, lse, selfcond, ws,
+                     stream=None):
+    """Finish a step from n_parts shard partials laid out back to back in `partials`."""
+    check("dg_denoise_merge", lib().dg_denoise_merge(
+        ctypes.byref(p), int(step), int(n_parts), _ptr(partials), _ptr(seeds), _ptr(tokens), _ptr(entropy),
+        _ptr(argmax), _ptr(accept), _ptr(lse), _ptr(selfcond), ws.ptr, ws.nbytes, _stream(stream)))
+
+
 def dg_stub_hidden(p, step, gain, noise, seeds, E, tokens, h, ws, stream=None):
     check("dg_stub_hidden", lib().dg_stub_hidden(ctypes.byref(p), int(step), float(gain), float(noise),
                                                  _ptr(seeds), _ptr(E), _ptr(tokens), _ptr(h), ws.ptr, ws.nbytes,
@@ -172,19 +195,21 @@ def decode_batch(p, W, E, seeds, gain=1.0, noise=0.1, hidden_fn=None, ws=None, b
     return bufs.argmax.view(C, p.canvas_len).clone(), stop_step
 
 
-def decode_block_ar(p1, W, E, n_blocks, seed0=0, gain=1.0, noise=0.1):
+def decode_block_ar(p1, W, E, n_blocks, seed0=0, gain=1.0, noise=0.1, on_step=None):
     """Block-autoregressive decoding: n_blocks canvases of 256 tokens one after another.
 
     p1 describes one canvas (n_canvas = 1); canvas b uses seed seed0 + b.  The
-    committed block of each canvas is appended to the output.  Returns (tokens
-    [n_blocks * 256] int32, per-block stop steps).
+    committed block of each canvas is appended to the output.  on_step(b, s, bufs),
+    if given, sees every step's buffers.  Returns (tokens [n_blocks * 256] int32,
+    per-block stop steps).
     """
     ws = Workspace(p1, W.device)
     bufs = StepBuffers(p1, W.device)
     out, steps = [], []
     for b in range(n_blocks):
         seeds = torch.tensor([seed0 + b], dtype=torch.int64, device=W.device)
-        committed, st = decode_batch(p1, W, E, seeds, gain, noise, ws=ws, bufs=bufs)
+        cb = None if on_step is None else (lambda s, bf, b=b: on_step(b, s, bf))
+        committed, st = decode_batch(p1, W, E, seeds, gain, noise, ws=ws, bufs=bufs, on_step=cb)
         out.append(committed.view(-1))
         steps.append(st[0])
     return torch.cat(out), steps

@@ -11,7 +11,8 @@ DG_OK, DG_EINVAL, DG_ECUDA, DG_EUNSUPPORTED, DG_ETIMEOUT, DG_ENOMEM = 0, -1, -2,
 # every symbol include/dg.h declares
 EXPORTS = ("dg_params_default", "dg_temperature", "dg_workspace_size", "dg_canvas_init", "dg_denoise_step",
            "dg_stop_check", "dg_stub_hidden", "dg_status_string", "dg_last_launch_count", "dg_plan",
-           "dg_profile_enable", "dg_profile_collect", "dg_denoise_stats_noalloc", "dg_debug_set_error")
+           "dg_profile_enable", "dg_profile_collect", "dg_denoise_stats_noalloc", "dg_debug_set_error",
+           "dg_partial_bytes", "dg_denoise_partial", "dg_denoise_merge")
 
 
 class DgParams(ctypes.Structure):
@@ -65,6 +66,12 @@ def lib():
         L.dg_plan.restype = i32
         L.dg_denoise_stats_noalloc.argtypes = [P, i32, vp, vp, vp, vp, vp, vp, vp, vp]
         L.dg_denoise_stats_noalloc.restype = i32
+        L.dg_partial_bytes.argtypes = [P]
+        L.dg_partial_bytes.restype = sz
+        L.dg_denoise_partial.argtypes = [P, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.dg_denoise_partial.restype = i32
+        L.dg_denoise_merge.argtypes = [P, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.dg_denoise_merge.restype = i32
         L.dg_profile_enable.argtypes = [i32]
         L.dg_profile_enable.restype = i32
         L.dg_profile_collect.argtypes = [ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_float),

@@ -8,7 +8,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdg.so")
 SOURCES = ["dg_api.cu", "dg_fused.cu", "dg_small.cu", "dg_noalloc.cu"]
-HEADERS = ["dg_common.cuh", "dg_fused.h", "dg_sm100.cuh", os.path.join("..", "..", "include", "dg.h")]
+HEADERS = ["dg_common.cuh", "dg_fused.h", "dg_host.h", "dg_sm100.cuh", os.path.join("..", "..", "include", "dg.h")]
 
 
 def nvcc_path():

@@ -11,12 +11,17 @@
 #include "../../include/dg.h"
 #include "dg_common.cuh"
 #include "dg_fused.h"
+#include "dg_host.h"
 
 using namespace dg;
+
+namespace dg {
+namespace host {
 
 namespace {
 
 constexpr int kFusedSmem = kFusedSmemBytes;
+constexpr int kMaxDevices = 64;
 thread_local int g_last_launches = 0;
 
 // Event pairs recorded around fused-kernel launches while profiling is enabled.
@@ -37,9 +42,50 @@ void profile_release() {
     g_prof.on = false;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+// Per-device set-up state: the shared-memory attribute of the fused kernels and
+// the number of CTA pairs resident at once (both belong to one device).
+std::mutex g_dev_mu;
+bool g_attr_done[kMaxDevices];
+int g_pairs[kMaxDevices];
+
+bool current_device(int* dev) {
+    return cudaGetDevice(dev) == cudaSuccess && *dev >= 0 && *dev < kMaxDevices;
+}
+
+// Caller holds g_dev_mu; `dev` is the current device.
+bool attr_set_locked(int dev) {
+    if (g_attr_done[dev]) return true;
+    if (cudaFuncSetAttribute(dg_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(dg_fused_sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem) !=
+            cudaSuccess)
+        return false;
+    g_attr_done[dev] = true;
+    return true;
+}
+
+bool params_ok(const dg_params* p) {
+    if (!p) return false;
+    if (p->n_canvas < 1 || p->n_canvas > kMaxCanvas) return false;
+    if (p->canvas_len != kCanvas) return false;
+    if (p->vocab < kBV || p->vocab % kBV != 0) return false;
+    if (p->hidden < 128 || p->hidden % 128 != 0) return false;
+    if (p->max_steps < 1) return false;
+    if (!(p->t_start > 0.f) || !(p->t_end > 0.f)) return false;
+    if (p->stability < 0) return false;
+    if (p->accept_mode != 0 && p->accept_mode != 1) return false;
+    if (p->accept_rule != 0 && p->accept_rule != 1) return false;
+    return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <class T>
+T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+}  // namespace
 
 EncodeTiledFn encode_fn() {
     static EncodeTiledFn fn = nullptr;
@@ -54,6 +100,19 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+bool encode_blocks_3d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                      uint32_t box_blocks) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || cols % 64 != 0) return false;
+    cuuint64_t dims[3] = {64, rows, cols / 64};
+    cuuint64_t strides[2] = {cols * 2, 128};
+    cuuint32_t box[3] = {64, box_rows, box_blocks};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int device_sm_count() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
@@ -63,27 +122,18 @@ int device_sm_count() {
 }
 
 bool fused_attr_set() {
-    static std::once_flag once;
-    static cudaError_t err = cudaSuccess;
-    std::call_once(once, [] {
-        err = cudaFuncSetAttribute(dg_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem);
-        if (err == cudaSuccess)
-            err = cudaFuncSetAttribute(dg_fused_sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kFusedSmem);
-    });
-    return err == cudaSuccess;
+    int dev = 0;
+    if (!current_device(&dev)) return false;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    return attr_set_locked(dev);
 }
 
-// How many CTA pairs of the fused kernel can be resident at once on the current
-// device (a pair is a cluster of two CTAs, one CTA per SM).
 int resident_pairs() {
-    static int cache[64];
-    static std::mutex mu;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
-    std::lock_guard<std::mutex> lock(mu);
-    if (cache[dev] > 0) return cache[dev];
-    if (!fused_attr_set()) return -1;
+    if (!current_device(&dev)) return -1;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (g_pairs[dev] > 0) return g_pairs[dev];
+    if (!attr_set_locked(dev)) return -1;
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(2 * 64);
@@ -98,26 +148,10 @@ int resident_pairs() {
     cfg.numAttrs = 1;
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, dg_fused_kernel, &cfg) != cudaSuccess || n <= 0) return -1;
-    cache[dev] = n;
+    g_pairs[dev] = n;
     return n;
 }
 
-bool params_ok(const dg_params* p) {
-    if (!p) return false;
-    if (p->n_canvas < 1 || p->n_canvas > kMaxCanvas) return false;
-    if (p->canvas_len != kCanvas) return false;
-    if (p->vocab < kBV || p->vocab % kBV != 0) return false;
-    if (p->hidden < 64 || p->hidden % 64 != 0) return false;
-    if (p->max_steps < 1) return false;
-    if (!(p->t_start > 0.f) || !(p->t_end > 0.f)) return false;
-    if (p->stability < 0) return false;
-    if (p->accept_mode != 0 && p->accept_mode != 1) return false;
-    if (p->accept_rule != 0 && p->accept_rule != 1) return false;
-    return true;
-}
-
-// Returns DG_OK and fills `pl`, or the reason the shape is not handled.
-// `pairs` is the number of CTA pairs resident at once.
 dg_status make_plan(const dg_params* p, int pairs, Plan* pl) {
     if (!params_ok(p)) return DG_EINVAL;
     int slice = 0;
@@ -155,27 +189,149 @@ dg_status make_plan(const dg_params* p, int pairs, Plan* pl) {
     return DG_OK;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-// 3-D view {64 columns, rows, cols/64 column blocks} of a row-major bf16 matrix:
-// one box of {64, box_rows, box_blocks} fills box_blocks consecutive 128-byte
-// swizzle atoms (the layout the UMMA descriptors use: K-major for h and W,
-// MN-major for P^T and E).
-bool encode_blocks_3d(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                      uint32_t box_rows, uint32_t box_blocks) {
-    if (!enc || cols % 64 != 0) return false;
-    cuuint64_t dims[3] = {64, rows, cols / 64};
-    cuuint64_t strides[2] = {cols * 2, 128};
-    cuuint32_t box[3] = {64, box_rows, box_blocks};
-    cuuint32_t es[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+dg_status plan_current_device(const dg_params* p, Plan* pl) {
+    const int pairs = resident_pairs();
+    if (pairs <= 0) return DG_ECUDA;
+    return make_plan(p, pairs, pl);
 }
 
-template <class T>
-T* at(void* ws, size_t off) {
-    return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+void set_last_launches(int n) { g_last_launches = n; }
+
+PartialLayout partial_layout(int N, int d) {
+    PartialLayout P{};
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t a = o;
+        o = align_up(o + bytes, 256);
+        return a;
+    };
+    P.stats = take(sizeof(float4) * static_cast<size_t>(N));
+    P.idx = take(sizeof(int32_t) * static_cast<size_t>(N));
+    P.skey = take(sizeof(float) * static_cast<size_t>(N));
+    P.sidx = take(sizeof(int32_t) * static_cast<size_t>(N));
+    P.o = take(sizeof(float) * static_cast<size_t>(N) * d);
+    P.total = o;
+    return P;
+}
+
+dg_status launch_fused_and_combine(const dg_params* p, const Plan& pl, const Layout& L, void* ws, int step,
+                                   const PassIO& io, cudaStream_t s) {
+    if (!fused_attr_set()) return DG_ECUDA;
+    const float T = dg_temperature(p, step);
+    FusedArgs fa;
+    std::memset(&fa, 0, sizeof(fa));
+    const uint64_t prow_total = static_cast<uint64_t>(pl.n_groups) * 2 * pl.group * kCanvas;
+    if (!encode_blocks_3d(&fa.map_h, io.h, pl.N, pl.d, kTileM, kKChunk / 64) ||
+        !encode_blocks_3d(&fa.map_w, io.W, io.vocab_rows, pl.d, kBV / 2, kKChunk / 64) ||
+        !encode_blocks_3d(&fa.map_e, io.E, io.vocab_rows, pl.d, kVChunk, pl.slice / 128) ||
+        !encode_blocks_3d(&fa.map_p, at<void>(ws, L.pbuf), prow_total, kCanvas, kVChunk, 2))
+        return DG_ECUDA;
+    int32_t* stop = at<int32_t>(ws, L.stop);
+    fa.stop = stop;
+    fa.counters = at<uint32_t>(ws, L.counters);
+    fa.rowmax = at<float>(ws, L.rowmax);
+    fa.pbuf = at<__nv_bfloat16>(ws, L.pbuf);
+    fa.stats = at<float4>(ws, L.stats);
+    fa.stat_idx = at<int32_t>(ws, L.stat_idx);
+    fa.opart = at<float>(ws, L.opart);
+    fa.err = at<int>(ws, L.err);
+    fa.seeds = io.seeds;
+    fa.skey = at<float>(ws, L.skey);
+    fa.sidx = at<int32_t>(ws, L.sidx);
+    fa.step = step;
+    fa.C = pl.C;
+    fa.V = io.vocab_rows;
+    fa.vocab_offset = io.vocab_offset;
+    fa.d = pl.d;
+    fa.G = pl.group;
+    fa.keep_w_stages = io.E == io.W ? (pl.d / kKChunk) * kKeepWTenths / 10 : 0;
+    fa.slice = pl.slice;
+    fa.n_groups = pl.n_groups;
+    fa.steps_per_tile = (io.vocab_rows + pl.group * kBV - 1) / (pl.group * kBV);
+    fa.max_seg = pl.max_seg;
+    fa.scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
+
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(2 * pl.n_groups * pl.group);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kFusedSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;   // CTA pairs
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const bool prof = g_prof.on && g_prof.used < g_prof.max_records;
+    if (prof && cudaEventRecord(g_prof.start[g_prof.used], s) != cudaSuccess) return DG_ECUDA;
+    if (cudaLaunchKernelEx(&cfg, p->accept_mode == 1 ? dg_fused_sample_kernel : dg_fused_kernel, fa) != cudaSuccess)
+        return DG_ECUDA;
+    if (prof) {
+        if (cudaEventRecord(g_prof.stop[g_prof.used], s) != cudaSuccess) return DG_ECUDA;
+        ++g_prof.used;
+    }
+
+    CombineArgs ca;
+    std::memset(&ca, 0, sizeof(ca));
+    ca.stop = stop;
+    ca.err = fa.err;
+    ca.counters = fa.counters;
+    ca.stats = fa.stats;
+    ca.stat_idx = fa.stat_idx;
+    ca.skey = fa.skey;
+    ca.sidx = fa.sidx;
+    ca.accept_mode = p->accept_mode;
+    ca.accept_rule = p->accept_rule;
+    ca.kept = at<int32_t>(ws, L.kept);
+    ca.opart = fa.opart;
+    ca.entropy = io.entropy;
+    ca.argmax = io.argmax;
+    ca.lse = io.lse;
+    ca.selfcond = io.selfcond;
+    if (io.partial) {
+        const PartialLayout P = partial_layout(pl.N, pl.d);
+        uint8_t* base = static_cast<uint8_t*>(io.partial);
+        ca.part_stats = reinterpret_cast<float4*>(base + P.stats);
+        ca.part_idx = reinterpret_cast<int32_t*>(base + P.idx);
+        ca.part_skey = reinterpret_cast<float*>(base + P.skey);
+        ca.part_sidx = reinterpret_cast<int32_t*>(base + P.sidx);
+        ca.part_o = reinterpret_cast<float*>(base + P.o);
+    }
+    ca.C = pl.C;
+    ca.d = pl.d;
+    ca.G = pl.group;
+    ca.n_groups = pl.n_groups;
+    ca.steps_per_tile = fa.steps_per_tile;
+    ca.max_seg = pl.max_seg;
+    ca.seeds = io.seeds;
+    ca.tokens = io.tokens;
+    ca.accept = io.accept;
+    ca.bound = p->eb_bound;
+    ca.step = step;
+    ca.V = pl.V;
+    dg_combine_kernel<<<combine_grid(pl.N, pl.d), 256, 0, s>>>(ca);
+    if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
+    return DG_OK;
+}
+
+}  // namespace host
+}  // namespace dg
+
+using namespace dg::host;
+
+namespace {
+
+dg_status launch_stop(const dg_params* p, const Plan& pl, const Layout& L, void* ws, int step,
+                      const uint64_t* seeds_dev, int32_t* tokens_dev, const float* entropy_dev,
+                      const int32_t* argmax_dev, uint8_t* accept_dev, cudaStream_t s) {
+    GroupAcceptArgs ga{p->accept_rule, p->eb_bound, at<int32_t>(ws, L.kept), seeds_dev, tokens_dev, accept_dev,
+                       pl.V};
+    dg_stop_kernel<<<pl.C, kCanvas, 0, s>>>(entropy_dev, argmax_dev, at<int32_t>(ws, L.prev_argmax),
+                                            at<int32_t>(ws, L.stable), at<int32_t>(ws, L.stop), p->stop_thresh,
+                                            p->stability, step, ga);
+    return cudaGetLastError() == cudaSuccess ? DG_OK : DG_ECUDA;
 }
 
 }  // namespace
@@ -225,10 +381,8 @@ const char* dg_status_string(dg_status s) {
 int dg_last_launch_count(void) { return g_last_launches; }
 
 dg_status dg_plan(const dg_params* p, int* group, int* n_groups, int* slice_cols) {
-    const int pairs = resident_pairs();
-    if (pairs <= 0) return DG_ECUDA;
     Plan pl;
-    dg_status st = make_plan(p, pairs, &pl);
+    const dg_status st = plan_current_device(p, &pl);
     if (st != DG_OK) return st;
     if (group) *group = pl.group;
     if (n_groups) *n_groups = pl.n_groups;
@@ -237,20 +391,16 @@ dg_status dg_plan(const dg_params* p, int* group, int* n_groups, int* slice_cols
 }
 
 size_t dg_workspace_size(const dg_params* p) {
-    const int pairs = resident_pairs();
-    if (pairs <= 0) return 0;
     Plan pl;
-    if (make_plan(p, pairs, &pl) != DG_OK) return 0;
+    if (plan_current_device(p, &pl) != DG_OK) return 0;
     return make_layout(pl).total;
 }
 
 dg_status dg_canvas_init(const dg_params* p, const uint64_t* seeds_dev, int32_t* tokens_dev, void* workspace_dev,
                          size_t workspace_bytes, void* stream) {
     g_last_launches = 0;
-    const int pairs = resident_pairs();
-    if (pairs <= 0) return DG_ECUDA;
     Plan pl;
-    dg_status st = make_plan(p, pairs, &pl);
+    const dg_status st = plan_current_device(p, &pl);
     if (st != DG_OK) return st;
     if (!seeds_dev || !tokens_dev || !workspace_dev) return DG_EINVAL;
     const Layout L = make_layout(pl);
@@ -272,10 +422,8 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
                           uint8_t* accept_dev, float* lse_dev, float* selfcond_dev, void* workspace_dev,
                           size_t workspace_bytes, void* stream) {
     g_last_launches = 0;
-    const int pairs = resident_pairs();
-    if (pairs <= 0) return DG_ECUDA;
     Plan pl;
-    dg_status st = make_plan(p, pairs, &pl);
+    const dg_status st = plan_current_device(p, &pl);
     if (st != DG_OK) return st;
     if (step < 1 || step > p->max_steps) return DG_EINVAL;
     if (!h_dev || !W_dev || !E_dev || !seeds_dev || !tokens_dev || !entropy_dev || !argmax_dev || !accept_dev ||
@@ -287,99 +435,112 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
     if (workspace_bytes < L.total) return DG_ENOMEM;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    if (!fused_attr_set()) return DG_ECUDA;
-
-    const float T = dg_temperature(p, step);
-    FusedArgs fa;
-    std::memset(&fa, 0, sizeof(fa));
-    const uint64_t prow_total = static_cast<uint64_t>(pl.n_groups) * 2 * pl.group * kCanvas;
-    if (!encode_blocks_3d(encode_fn(), &fa.map_h, h_dev, pl.N, pl.d, kTileM, kKChunk / 64) ||
-        !encode_blocks_3d(encode_fn(), &fa.map_w, W_dev, pl.V, pl.d, kBV / 2, kKChunk / 64) ||
-        !encode_blocks_3d(encode_fn(), &fa.map_e, E_dev, pl.V, pl.d, kVChunk, pl.slice / 128) ||
-        !encode_blocks_3d(encode_fn(), &fa.map_p, at<void>(workspace_dev, L.pbuf), prow_total, kCanvas, kVChunk, 2))
-        return DG_ECUDA;
-    int32_t* stop = at<int32_t>(workspace_dev, L.stop);
-    fa.stop = stop;
-    fa.counters = at<uint32_t>(workspace_dev, L.counters);
-    fa.rowmax = at<float>(workspace_dev, L.rowmax);
-    fa.pbuf = at<__nv_bfloat16>(workspace_dev, L.pbuf);
-    fa.stats = at<float4>(workspace_dev, L.stats);
-    fa.stat_idx = at<int32_t>(workspace_dev, L.stat_idx);
-    fa.opart = at<float>(workspace_dev, L.opart);
-    fa.err = at<int>(workspace_dev, L.err);
-    fa.seeds = seeds_dev;
-    fa.skey = at<float>(workspace_dev, L.skey);
-    fa.sidx = at<int32_t>(workspace_dev, L.sidx);
-    fa.step = step;
-    fa.C = pl.C;
-    fa.V = pl.V;
-    fa.d = pl.d;
-    fa.G = pl.group;
-    fa.keep_w_stages = E_dev == W_dev ? (pl.d / kKChunk) * kKeepWTenths / 10 : 0;
-    fa.slice = pl.slice;
-    fa.n_groups = pl.n_groups;
-    fa.steps_per_tile = pl.steps_per_tile;
-    fa.max_seg = pl.max_seg;
-    fa.scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
-
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(2 * pl.n_groups * pl.group);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kFusedSmem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;   // CTA pairs
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const bool prof = g_prof.on && g_prof.used < g_prof.max_records;
-    if (prof && cudaEventRecord(g_prof.start[g_prof.used], s) != cudaSuccess) return DG_ECUDA;
-    if (cudaLaunchKernelEx(&cfg, p->accept_mode == 1 ? dg_fused_sample_kernel : dg_fused_kernel, fa) != cudaSuccess)
-        return DG_ECUDA;
-    if (prof) {
-        if (cudaEventRecord(g_prof.stop[g_prof.used], s) != cudaSuccess) return DG_ECUDA;
-        ++g_prof.used;
-    }
-
-    CombineArgs ca;
-    ca.stop = stop;
-    ca.counters = fa.counters;
-    ca.stats = fa.stats;
-    ca.stat_idx = fa.stat_idx;
-    ca.skey = fa.skey;
-    ca.sidx = fa.sidx;
-    ca.accept_mode = p->accept_mode;
-    ca.accept_rule = p->accept_rule;
-    ca.kept = at<int32_t>(workspace_dev, L.kept);
-    ca.opart = fa.opart;
-    ca.entropy = entropy_dev;
-    ca.argmax = argmax_dev;
-    ca.lse = lse_dev;
-    ca.selfcond = selfcond_dev;
-    ca.C = pl.C;
-    ca.d = pl.d;
-    ca.G = pl.group;
-    ca.n_groups = pl.n_groups;
-    ca.steps_per_tile = pl.steps_per_tile;
-    ca.max_seg = pl.max_seg;
-    ca.seeds = seeds_dev;
-    ca.tokens = tokens_dev;
-    ca.accept = accept_dev;
-    ca.bound = p->eb_bound;
-    ca.step = step;
-    ca.V = pl.V;
-    dg_combine_kernel<<<combine_grid(pl.N, pl.d), 256, 0, s>>>(ca);
-    if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
-
-    GroupAcceptArgs ga{p->accept_rule, p->eb_bound, ca.kept, seeds_dev, tokens_dev, accept_dev, pl.V};
-    dg_stop_kernel<<<pl.C, kCanvas, 0, s>>>(entropy_dev, argmax_dev, at<int32_t>(workspace_dev, L.prev_argmax),
-                                            at<int32_t>(workspace_dev, L.stable), stop, p->stop_thresh, p->stability,
-                                            step, ga);
-    if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
+    PassIO io{};
+    io.h = h_dev;
+    io.W = W_dev;
+    io.E = E_dev;
+    io.seeds = seeds_dev;
+    io.tokens = tokens_dev;
+    io.entropy = entropy_dev;
+    io.argmax = argmax_dev;
+    io.accept = accept_dev;
+    io.lse = lse_dev;
+    io.selfcond = selfcond_dev;
+    io.vocab_offset = 0;
+    io.vocab_rows = pl.V;
+    dg_status r = launch_fused_and_combine(p, pl, L, workspace_dev, step, io, s);
+    if (r != DG_OK) return r;
+    r = launch_stop(p, pl, L, workspace_dev, step, seeds_dev, tokens_dev, entropy_dev, argmax_dev, accept_dev, s);
+    if (r != DG_OK) return r;
     g_last_launches = 3;
+    return DG_OK;
+}
+
+size_t dg_partial_bytes(const dg_params* p) {
+    if (!p || p->n_canvas < 1 || p->n_canvas > kMaxCanvas || p->canvas_len != kCanvas || p->hidden < 128 ||
+        p->hidden % 128 != 0)
+        return 0;
+    return partial_layout(p->n_canvas * kCanvas, p->hidden).total;
+}
+
+dg_status dg_denoise_partial(const dg_params* p, int step, int v_begin, int v_count, const void* h_dev,
+                             const void* W_shard_dev, const void* E_shard_dev, const uint64_t* seeds_dev,
+                             void* partial_dev, void* workspace_dev, size_t workspace_bytes, void* stream) {
+    g_last_launches = 0;
+    Plan pl;
+    dg_status st = plan_current_device(p, &pl);
+    if (st != DG_OK) return st;
+    if (step < 1 || step > p->max_steps) return DG_EINVAL;
+    if (v_begin < 0 || v_count < kBV || v_begin % kBV != 0 || v_count % kBV != 0 ||
+        static_cast<long long>(v_begin) + v_count > p->vocab)
+        return DG_EINVAL;
+    if (!h_dev || !W_shard_dev || !E_shard_dev || !seeds_dev || !partial_dev || !workspace_dev) return DG_EINVAL;
+    if (!aligned16(h_dev) || !aligned16(W_shard_dev) || !aligned16(E_shard_dev) || !aligned16(partial_dev))
+        return DG_EINVAL;
+    const Layout L = make_layout(pl);
+    if (workspace_bytes < L.total) return DG_ENOMEM;
+    PassIO io{};
+    io.h = h_dev;
+    io.W = W_shard_dev;
+    io.E = E_shard_dev;
+    io.seeds = seeds_dev;
+    io.partial = partial_dev;
+    io.vocab_offset = v_begin;
+    io.vocab_rows = v_count;
+    st = launch_fused_and_combine(p, pl, L, workspace_dev, step, io, static_cast<cudaStream_t>(stream));
+    if (st != DG_OK) return st;
+    g_last_launches = 2;
+    return DG_OK;
+}
+
+dg_status dg_denoise_merge(const dg_params* p, int step, int n_parts, const void* partials_dev,
+                           const uint64_t* seeds_dev, int32_t* tokens_dev, float* entropy_dev, int32_t* argmax_dev,
+                           uint8_t* accept_dev, float* lse_dev, float* selfcond_dev, void* workspace_dev,
+                           size_t workspace_bytes, void* stream) {
+    g_last_launches = 0;
+    Plan pl;
+    dg_status st = plan_current_device(p, &pl);
+    if (st != DG_OK) return st;
+    if (step < 1 || step > p->max_steps) return DG_EINVAL;
+    if (n_parts < 1 || n_parts > kMaxParts) return DG_EINVAL;
+    if (!partials_dev || !seeds_dev || !tokens_dev || !entropy_dev || !argmax_dev || !accept_dev || !workspace_dev)
+        return DG_EINVAL;
+    if (!aligned16(partials_dev) || (selfcond_dev && !aligned16(selfcond_dev))) return DG_EINVAL;
+    const Layout L = make_layout(pl);
+    if (workspace_bytes < L.total) return DG_ENOMEM;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const PartialLayout P = partial_layout(pl.N, pl.d);
+    MergeArgs ma;
+    std::memset(&ma, 0, sizeof(ma));
+    ma.partials = static_cast<const uint8_t*>(partials_dev);
+    ma.part_bytes = P.total;
+    ma.off_stats = P.stats;
+    ma.off_idx = P.idx;
+    ma.off_skey = P.skey;
+    ma.off_sidx = P.sidx;
+    ma.off_o = P.o;
+    ma.n_parts = n_parts;
+    ma.stop = at<int32_t>(workspace_dev, L.stop);
+    ma.accept_mode = p->accept_mode;
+    ma.accept_rule = p->accept_rule;
+    ma.kept = at<int32_t>(workspace_dev, L.kept);
+    ma.entropy = entropy_dev;
+    ma.argmax = argmax_dev;
+    ma.lse = lse_dev;
+    ma.selfcond = selfcond_dev;
+    ma.seeds = seeds_dev;
+    ma.tokens = tokens_dev;
+    ma.accept = accept_dev;
+    ma.bound = p->eb_bound;
+    ma.step = step;
+    ma.V = pl.V;
+    ma.N = pl.N;
+    ma.d = pl.d;
+    dg_merge_kernel<<<combine_grid(pl.N, pl.d), 256, 0, s>>>(ma);
+    if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
+    st = launch_stop(p, pl, L, workspace_dev, step, seeds_dev, tokens_dev, entropy_dev, argmax_dev, accept_dev, s);
+    if (st != DG_OK) return st;
+    g_last_launches = 2;
     return DG_OK;
 }
 
@@ -426,10 +587,8 @@ dg_status dg_profile_collect(int* n_records, float* mean_ms, float* total_ms) {
 
 dg_status dg_stop_check(const dg_params* p, void* workspace_dev, size_t workspace_bytes, int32_t* stop_flags_host,
                         int32_t* stable_host, int* n_stopped_host, void* stream) {
-    const int pairs = resident_pairs();
-    if (pairs <= 0) return DG_ECUDA;
     Plan pl;
-    dg_status st = make_plan(p, pairs, &pl);
+    const dg_status st = plan_current_device(p, &pl);
     if (st != DG_OK) return st;
     if (!workspace_dev) return DG_EINVAL;
     const Layout L = make_layout(pl);
@@ -459,10 +618,8 @@ dg_status dg_stop_check(const dg_params* p, void* workspace_dev, size_t workspac
 
 dg_status dg_debug_set_error(const dg_params* p, void* workspace_dev, size_t workspace_bytes, int32_t code,
                              void* stream) {
-    const int pairs = resident_pairs();
-    if (pairs <= 0) return DG_ECUDA;
     Plan pl;
-    dg_status st = make_plan(p, pairs, &pl);
+    const dg_status st = plan_current_device(p, &pl);
     if (st != DG_OK) return st;
     if (!workspace_dev) return DG_EINVAL;
     const Layout L = make_layout(pl);
@@ -478,10 +635,8 @@ dg_status dg_stub_hidden(const dg_params* p, int step, float gain, float noise, 
                          const void* E_dev, const int32_t* tokens_dev, void* h_dev, void* workspace_dev,
                          size_t workspace_bytes, void* stream) {
     g_last_launches = 0;
-    const int pairs = resident_pairs();
-    if (pairs <= 0) return DG_ECUDA;
     Plan pl;
-    dg_status st = make_plan(p, pairs, &pl);
+    const dg_status st = plan_current_device(p, &pl);
     if (st != DG_OK) return st;
     if (step < 1 || step > p->max_steps) return DG_EINVAL;
     if (!seeds_dev || !E_dev || !tokens_dev || !h_dev || !workspace_dev) return DG_EINVAL;

@@ -17,6 +17,7 @@ constexpr int kKChunk = 128;      // hidden columns per pipeline stage of the lo
 constexpr int kVChunk = 128;      // vocabulary rows per pipeline stage of the self-conditioning GEMM
 constexpr int kMaxSlice = 256;    // widest self-conditioning column slice a CTA pair keeps in TMEM
 constexpr int kMaxCanvas = 256;   // canvases per call (the fused kernel keeps the active list in shared memory)
+constexpr int kMaxParts = 64;     // vocabulary shards one dg_denoise_merge call takes
 constexpr int kThreads = 256;     // threads of the fused kernel
 constexpr int kFusedStages = 3;   // TMA ring stages of the fused kernel
 constexpr int kFusedStageBytes = 64 * 1024;

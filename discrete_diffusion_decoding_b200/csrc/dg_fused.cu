@@ -504,7 +504,7 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                     __nv_bfloat16* pt = a.pbuf + static_cast<size_t>((g * 2 + (k & 1)) * G + r) * kBV * kCanvas;
                     const bool odd = lane & 1;
                     const int prow = crow & ~1;
-                    const int v0 = vocab0(t, r);
+                    const int v0 = vocab0(t, r) + a.vocab_offset;     // global vocabulary index of column 0
 #pragma unroll 1
                     for (int c0 = 0; c0 < kBV; c0 += 64) {
                         uint32_t v[64];
@@ -635,23 +635,68 @@ __global__ void __launch_bounds__(kThreads, 1) dg_fused_sample_kernel(const __gr
 }
 
 // ---------------------------------------------------------------------------
+// Finishing a position from its merged statistics (juhoplayground, entropy
+// bounded sampler; deep dive steps 4-5):
+//   H = ln L - ln2 * U / L;  LSE = ln2 * (M + log2 L);
+// then keep the argmax where H <= bound (in the sampled mode the Gumbel-max
+// sample), otherwise a uniform vocabulary token from Philox (tag 1, this step).
+// With the group rule only the kept token is stored (dg_stop_kernel decides).
+// A position whose statistics come from a pass that recorded an error is
+// poisoned: H and LSE NaN, argmax -1, re-noised, never accepted.
+struct Finish {
+    float* entropy;
+    int32_t* argmax;
+    float* lse;
+    int32_t* tokens;
+    uint8_t* accept;
+    int32_t* kept;
+    const uint64_t* seeds;
+    float bound;
+    int step, V, accept_mode, accept_rule;
+};
+
+__device__ void finish_position(const Finish& f, int n, int c, int crow, float M, float L, float U, int bidx,
+                                int sidx, bool bad) {
+    const float ln2 = 0.69314718055994531f;
+    float H = logf(L) - ln2 * (U / L);
+    float lse = ln2 * (M + log2f(L));
+    if (bad) {
+        H = __int_as_float(0x7fc00000);
+        lse = H;
+        bidx = -1;
+    }
+    f.entropy[n] = H;
+    f.argmax[n] = bidx;
+    if (f.lse) f.lse[n] = lse;
+    if (!f.tokens) return;
+    const int32_t renoise = philox_token(f.seeds[c], static_cast<uint32_t>(crow), static_cast<uint32_t>(f.step),
+                                         static_cast<uint32_t>(c), kTagRenoise, static_cast<uint32_t>(f.V));
+    const int32_t keep = f.accept_mode == 1 ? sidx : bidx;
+    if (f.accept_rule == 1) {
+        f.kept[n] = bad ? renoise : keep;          // accepted by groups in dg_stop_kernel
+    } else {
+        const bool acc = !bad && H <= f.bound;
+        f.tokens[n] = acc ? keep : renoise;
+        f.accept[n] = acc ? 1 : 0;
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Split-vocabulary combine: one CTA per (active position, block of 1024
 // self-conditioning columns).  Merges the partial statistics of every (piece,
 // pair) covering the position's canvas:
 //   M = max m_s;  L = sum_s 2^(m_s-M) sum_r l;  U = sum_s 2^(m_s-M) (sum_r u + (m_s-M) sum_r l)
-//   H = ln L - ln2 * U / L;  LSE = ln2 * (M + log2 L);  argmax = best raw logit, smallest index;
-//   sc = sum_s 2^(m_s-M) O_s / L.
-// The column-block-0 CTA of a position also writes H / argmax / LSE and applies
-// the entropy-bounded sampler to it (juhoplayground, entropy bounded sampler;
-// deep dive steps 4-5): keep the argmax where H <= bound (in the sampled mode the
-// Gumbel-max sample: the largest key over all pieces, smallest index on a tie),
-// otherwise a uniform vocabulary token from Philox (tag 1, this step).  CTA (0, 0)
-// also clears the fused kernel's group counters for its next launch.
+//   argmax = best raw logit, smallest index;  sc = sum_s 2^(m_s-M) O_s / L.
+// The column-block-0 CTA of a position finishes it (finish_position).  In shard
+// mode (a vocabulary shard of a split head) it writes the merged statistics and
+// the unnormalised numerator sum_s 2^(m_s-M) O_s instead.  CTA (0, 0) also clears
+// the fused kernel's group counters for its next launch.
 __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
     __shared__ float sh_w[kMaxSlotsPerTile];
     __shared__ int sh_slot[kMaxSlotsPerTile];
     __shared__ int n_slots_s;
     __shared__ float sh_L;
+    __shared__ int sh_bad;
     __shared__ int sh_active_rank;
     __shared__ int sh_n_active;
     __shared__ int sh_skip;
@@ -666,6 +711,7 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
     }
     if (tid == 0) {
         sh_skip = a.stop[c] != 0;
+        sh_bad = a.err != nullptr && *reinterpret_cast<const volatile int*>(a.err) != 0;
         int rank = 0, na = 0;
         for (int q = 0; q < a.C; ++q) {
             const int act = a.stop[q] == 0;
@@ -679,6 +725,7 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
     if (sh_skip) return;
     const int ct = sh_active_rank;
     const int T = a.steps_per_tile;
+    const bool bad = sh_bad != 0;
 
     if (tid < 32) {
         // warp 0: merge statistics over (slot, pair) entries.  The slots of this canvas's
@@ -757,31 +804,26 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
         }
         if (tid == 0) {
             sh_L = L;
-            if (head) {
-                const float ln2 = 0.69314718055994531f;
-                const float H = logf(L) - ln2 * (Uu / L);
-                a.entropy[n] = H;
-                a.argmax[n] = bidx;
-                if (a.lse) a.lse[n] = ln2 * (M + log2f(L));
-                if (a.tokens && a.accept_rule == 1) {
-                    a.kept[n] = a.accept_mode == 1 ? sidx : bidx;     // accepted by groups in dg_stop_kernel
-                } else if (a.tokens) {
-                    const bool acc = H <= a.bound;
-                    a.tokens[n] = acc ? (a.accept_mode == 1 ? sidx : bidx)
-                                      : philox_token(a.seeds[c], static_cast<uint32_t>(crow),
-                                                     static_cast<uint32_t>(a.step), static_cast<uint32_t>(c),
-                                                     kTagRenoise, static_cast<uint32_t>(a.V));
-                    a.accept[n] = acc ? 1 : 0;
-                }
+            if (head && a.part_stats) {
+                const float nan = __int_as_float(0x7fc00000);
+                a.part_stats[n] = bad ? make_float4(nan, nan, nan, nan) : make_float4(M, L, Uu, best);
+                a.part_idx[n] = bad ? -1 : bidx;
+                a.part_skey[n] = skey;
+                a.part_sidx[n] = a.accept_mode == 1 ? sidx : -1;
+            } else if (head) {
+                const Finish f{a.entropy, a.argmax, a.lse, a.tokens, a.accept, a.kept, a.seeds, a.bound,
+                               a.step, a.V, a.accept_mode, a.accept_rule};
+                finish_position(f, n, c, crow, M, L, Uu, bidx, sidx, bad);
             }
         }
         for (int s = tid; s < ns; s += 32)
             sh_w[s] = exp2f(a.stats[(static_cast<size_t>(sh_slot[s]) * a.G) * kCanvas + crow].x - M);
     }
     __syncthreads();
-    if (a.selfcond == nullptr) return;
+    float* out = a.part_o ? a.part_o : a.selfcond;
+    if (out == nullptr) return;
     const int ns = n_slots_s;
-    const float invL = 1.f / sh_L;
+    const float scale = bad ? __int_as_float(0x7fc00000) : (a.part_o ? 1.f : 1.f / sh_L);
     const int col_end = min(a.d, static_cast<int>(blockIdx.y + 1) * kCombineCols);
     for (int col = static_cast<int>(blockIdx.y) * kCombineCols + tid * 4; col < col_end; col += blockDim.x * 4) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -795,10 +837,114 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
             acc.z = fmaf(w, o.z, acc.z);
             acc.w = fmaf(w, o.w, acc.w);
         }
+        *reinterpret_cast<float4*>(out + static_cast<size_t>(n) * a.d + col) =
+            make_float4(acc.x * scale, acc.y * scale, acc.z * scale, acc.w * scale);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Merge of vocabulary shards (a head split by vocabulary rows over several
+// devices, or several calls): the same LSE merge as the combine, over the shards'
+// partials instead of the pieces of one pass.  One CTA per (active position,
+// block of 1024 self-conditioning columns); warp 0 merges the statistics (one
+// lane per shard), then the position is finished as in the combine.  A shard
+// whose statistics are NaN (its pass recorded an error) poisons the position.
+__global__ void __launch_bounds__(256) dg_merge_kernel(const MergeArgs a) {
+    __shared__ float sh_w[kMaxParts];
+    __shared__ float sh_L;
+    __shared__ int sh_bad;
+    __shared__ int sh_skip;
+    const int n = blockIdx.x;
+    const int c = n / kCanvas;
+    const int crow = n % kCanvas;
+    const int tid = threadIdx.x;
+    const bool head = blockIdx.y == 0;
+    if (tid == 0) sh_skip = a.stop[c] != 0;
+    __syncthreads();
+    if (sh_skip) return;
+    auto stats_of = [&](int g) {
+        return reinterpret_cast<const float4*>(a.partials + static_cast<size_t>(g) * a.part_bytes + a.off_stats)[n];
+    };
+    if (tid < 32) {
+        float M = -INFINITY;
+        bool bad = false;
+        for (int g = tid; g < a.n_parts; g += 32) {
+            const float m = stats_of(g).x;
+            bad |= m != m;
+            M = fmaxf(M, m);
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        bad = __any_sync(0xffffffffu, bad);
+        float L = 0.f, U = 0.f, best = -INFINITY, skey = -INFINITY;
+        int bidx = 0x7fffffff, sidx = 0x7fffffff;
+        for (int g = tid; g < a.n_parts; g += 32) {
+            const uint8_t* base = a.partials + static_cast<size_t>(g) * a.part_bytes;
+            const float4 st = stats_of(g);
+            const int idx = reinterpret_cast<const int32_t*>(base + a.off_idx)[n];
+            const float w = exp2f(st.x - M);
+            L += w * st.y;
+            U += w * (st.z + (st.x - M) * st.y);
+            if (idx >= 0 && (st.w > best || (st.w == best && idx < bidx))) {
+                best = st.w;
+                bidx = idx;
+            }
+            if (a.accept_mode == 1) {
+                const float kk = reinterpret_cast<const float*>(base + a.off_skey)[n];
+                const int ki = reinterpret_cast<const int32_t*>(base + a.off_sidx)[n];
+                if (ki >= 0 && (kk > skey || (kk == skey && ki < sidx))) {
+                    skey = kk;
+                    sidx = ki;
+                }
+            }
+            sh_w[g] = w;
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) {
+            L += __shfl_xor_sync(0xffffffffu, L, off);
+            U += __shfl_xor_sync(0xffffffffu, U, off);
+            const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
+            if (ob > best || (ob == best && oi < bidx)) {
+                best = ob;
+                bidx = oi;
+            }
+            const float ok = __shfl_xor_sync(0xffffffffu, skey, off);
+            const int oki = __shfl_xor_sync(0xffffffffu, sidx, off);
+            if (ok > skey || (ok == skey && oki < sidx)) {
+                skey = ok;
+                sidx = oki;
+            }
+        }
+        if (tid == 0) {
+            sh_L = L;
+            sh_bad = bad;
+            if (head) {
+                const Finish f{a.entropy, a.argmax, a.lse, a.tokens, a.accept, a.kept, a.seeds, a.bound,
+                               a.step, a.V, a.accept_mode, a.accept_rule};
+                finish_position(f, n, c, crow, M, L, U, bidx, sidx, bad);
+            }
+        }
+    }
+    __syncthreads();
+    if (a.selfcond == nullptr) return;
+    const float scale = sh_bad ? __int_as_float(0x7fc00000) : 1.f / sh_L;
+    const int col_end = min(a.d, static_cast<int>(blockIdx.y + 1) * kCombineCols);
+    for (int col = static_cast<int>(blockIdx.y) * kCombineCols + tid * 4; col < col_end; col += blockDim.x * 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int g = 0; g < a.n_parts; ++g) {
+            const float* o = reinterpret_cast<const float*>(a.partials + static_cast<size_t>(g) * a.part_bytes +
+                                                            a.off_o);
+            const float4 v = *reinterpret_cast<const float4*>(o + static_cast<size_t>(n) * a.d + col);
+            const float w = sh_w[g];
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+        }
         *reinterpret_cast<float4*>(a.selfcond + static_cast<size_t>(n) * a.d + col) =
-            make_float4(acc.x * invL, acc.y * invL, acc.z * invL, acc.w * invL);
+            make_float4(acc.x * scale, acc.y * scale, acc.z * scale, acc.w * scale);
     }
 }
 
 }  // namespace dg
-

@@ -30,6 +30,8 @@ struct FusedArgs {
     int32_t* sidx;
     int step;
     int C, V, d, G, slice, n_groups, steps_per_tile, max_seg;
+    int vocab_offset;    // vocabulary index of row 0 of W / E (a shard of the vocabulary; 0 otherwise):
+                         // added to the argmax and sample indices and to the sampled mode's chunk counter
     int keep_w_stages;   // E aliases W: the first keep_w_stages hidden-column stages of every W
                          // tile keep normal L2 priority, so the self-conditioning pass finds them
                          // there (0 when E is a separate matrix)
@@ -38,6 +40,7 @@ struct FusedArgs {
 
 struct CombineArgs {
     const int32_t* stop;
+    const int* err;          // the fused kernel's error word: when set, every output is poisoned (NaN, -1)
     uint32_t* counters;
     const float4* stats;
     const int32_t* stat_idx;
@@ -58,6 +61,33 @@ struct CombineArgs {
     float bound;
     int step, V;
     int C, d, G, n_groups, steps_per_tile, max_seg;
+    // shard mode (part_stats non-null): write the merged statistics of this vocabulary shard and
+    // its unnormalised self-conditioning numerator instead of finishing (no accept / re-noise)
+    float4* part_stats;      // [N] {m, l, u, best}: m absolute (log2 units), l and u relative to m
+    int32_t* part_idx;       // [N] argmax of the shard (vocabulary index)
+    float* part_skey;        // [N] best sampled key (accept_mode 1)
+    int32_t* part_sidx;      // [N] its vocabulary index
+    float* part_o;           // [N, d] sum_v 2^(y_v - m) E_v
+};
+
+// Merge of the partials of n_parts vocabulary shards (dg_denoise_merge), laid out
+// back to back, part_bytes apart, each as dg_host.h's PartialLayout.
+struct MergeArgs {
+    const uint8_t* partials;
+    size_t part_bytes, off_stats, off_idx, off_skey, off_sidx, off_o;
+    int n_parts;
+    const int32_t* stop;
+    int accept_mode, accept_rule;
+    int32_t* kept;
+    float* entropy;
+    int32_t* argmax;
+    float* lse;
+    float* selfcond;
+    const uint64_t* seeds;
+    int32_t* tokens;
+    uint8_t* accept;
+    float bound;
+    int step, V, N, d;
 };
 
 // Combine grid: one CTA per (position, block of kCombineCols self-conditioning columns).
@@ -67,6 +97,7 @@ inline dim3 combine_grid(int N, int d) { return dim3(N, (d + kCombineCols - 1) /
 __global__ void dg_fused_kernel(const __grid_constant__ FusedArgs a);          // argmax acceptance
 __global__ void dg_fused_sample_kernel(const __grid_constant__ FusedArgs a);   // + Gumbel-max sample
 __global__ void dg_combine_kernel(const CombineArgs a);
+__global__ void dg_merge_kernel(const MergeArgs a);
 
 // small kernels (dg_small.cu)
 __global__ void dg_init_kernel(const uint64_t* seeds, int32_t* tokens, int32_t* prev_argmax, int32_t* stable,

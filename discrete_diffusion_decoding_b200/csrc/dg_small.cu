@@ -41,7 +41,9 @@ __device__ void group_accept(const float* entropy, const GroupAcceptArgs& ga, in
     __shared__ unsigned long long key[kCanvas];
     __shared__ int n_acc;
     const int tid = threadIdx.x;
-    const float h = fmaxf(entropy[c * kCanvas + tid], 0.f);
+    // a NaN entropy (a position poisoned by a failed pass) sorts last and is never accepted
+    const float hv = entropy[c * kCanvas + tid];
+    const float h = hv != hv ? INFINITY : fmaxf(hv, 0.f);
     key[tid] = (static_cast<unsigned long long>(__float_as_uint(h)) << 32) | static_cast<unsigned>(tid);
     __syncthreads();
     for (int k = 2; k <= kCanvas; k <<= 1) {

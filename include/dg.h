@@ -31,7 +31,15 @@
  *    synchronises that stream.  Argument errors are reported before anything
  *    is launched.  Nothing throws across this boundary.
  *  - A wait inside a kernel that runs past its time limit records an error
- *    word in the workspace; the next dg_stop_check returns DG_ETIMEOUT.
+ *    word in the workspace; the next dg_stop_check returns DG_ETIMEOUT, and
+ *    until dg_canvas_init clears the word every step writes poisoned results
+ *    (entropy and log-sum-exp NaN, argmax -1, self-conditioning NaN, every
+ *    position re-noised and none accepted), so a failed pass cannot pass for a
+ *    result.
+ *  - Set-up per device: the first call on a device that needs the fused kernel's
+ *    grid (dg_workspace_size, dg_plan, dg_canvas_init, dg_denoise_step, ...)
+ *    raises the fused kernels' shared-memory limit on that device and queries
+ *    how many CTA pairs fit there; make it before capturing a stream.
  *  - Philox4x32-10 (Salmon et al., SC'11) keys: key = (lo32(seed_c), hi32(seed_c)),
  *    counter = (position within canvas, step, canvas index, tag); tag 0 canvas
  *    init (step 0), 1 re-noise, 2 stub target ids, 3 stub Gaussian noise.
@@ -59,10 +67,13 @@ typedef enum {
 /*
  * Sampler configuration.  Defaults from the deep dive's settings table:
  * max_steps 48, temperature 0.8 -> 0.4, entropy bound 0.1, stop threshold
- * 0.005, stability 2.  Supported shapes: canvas_len == 256; vocab a multiple of
- * 256 and < 2^31; hidden a multiple of 64 whose column slice width (hidden /
- * group) is a multiple of 64 and at most 256, with group <= the SM count;
- * 1 <= n_canvas <= 1024.
+ * 0.005, stability 2.  Supported shapes (each checked before anything is launched):
+ *   canvas_len == 256, 1 <= n_canvas <= 256, vocab >= 256 and a multiple of 256,
+ *   hidden >= 128 and a multiple of 128, max_steps >= 1, both temperatures > 0,
+ *   stability >= 0, accept_mode and accept_rule 0 or 1 (DG_EINVAL otherwise);
+ *   the column slice hidden / group must be a multiple of 128 and at most 256, and
+ *   group (hidden / slice) pairs of CTAs must fit on the device at once
+ *   (DG_EUNSUPPORTED otherwise; with group = 0 the widest such slice is chosen).
  */
 typedef struct {
     int n_canvas;       /* C: independent canvases processed together */
@@ -184,7 +195,9 @@ dg_status dg_stub_hidden(const dg_params* p, int step, float gain, float noise, 
 /* Static description of a status code. */
 const char* dg_status_string(dg_status s);
 
-/* Number of kernel launches the last dg_denoise_step on this thread issued. */
+/* Number of kernel launches the last launching call (dg_canvas_init, dg_denoise_step,
+ * dg_stub_hidden, dg_denoise_partial, dg_denoise_merge, dg_denoise_stats_noalloc) on this
+ * host thread issued; 0 when it failed before launching. */
 int dg_last_launch_count(void);
 
 /*
@@ -221,11 +234,57 @@ dg_status dg_profile_collect(int* n_records, float* mean_ms, float* total_ms);
  * that point), so make that first call before capturing a stream.  All calls on a device share the array
  * and the call clears what must start at zero; calls whose GPU work overlaps
  * (different streams, or no ordering between them) race on it.  An in-kernel
- * wait that runs out is not reported by this call.
+ * wait that runs out makes this call's results poisoned (every entropy and
+ * log-sum-exp NaN, every argmax -1, self-conditioning NaN); the status it
+ * returns only covers the launches.
  */
 dg_status dg_denoise_stats_noalloc(const dg_params* p, int step, const void* h_dev, const void* W_dev,
                                    const void* E_dev, float* entropy_dev, int32_t* argmax_dev, float* lse_dev,
                                    float* selfcond_dev, void* stream);
+
+/*
+ * Vocabulary-parallel split (one head split by vocabulary rows over several
+ * devices or several calls).  The pages describe no multi-device scheme; the
+ * split follows from the log-sum-exp merge that the fused pass already uses
+ * between its pieces: every shard's statistics and self-conditioning numerator
+ * merge exactly, whatever the split.
+ *
+ * dg_partial_bytes: bytes of one shard's partial for p (0 if p is invalid).  A
+ * partial holds, per position, the shard's maximum scaled logit m (log2 units),
+ * l = sum e, u = sum e (z - m), the best raw logit with its index, the sampled
+ * key with its index (accept_mode 1), and the numerator sum_v 2^(z_v - m) E_v
+ * [N, d] fp32.  Partials of several shards are laid out back to back (what an
+ * all-gather of one buffer per shard produces).
+ */
+size_t dg_partial_bytes(const dg_params* p);
+
+/*
+ * The fused pass over vocabulary rows [v_begin, v_begin + v_count) only:
+ * W_shard_dev and E_shard_dev point at those rows ([v_count, d] bf16, row-major);
+ * p describes the whole head (p->vocab is the full vocabulary).  Writes the
+ * shard's partial to partial_dev (dg_partial_bytes(p) bytes, 16-byte aligned).
+ * v_begin and v_count are multiples of 256, v_count >= 256 and the range lies in
+ * [0, p->vocab) (DG_EINVAL otherwise).  Canvases whose stop flag is set in the
+ * workspace are skipped.  Asynchronous on `stream`; two launches.
+ */
+dg_status dg_denoise_partial(const dg_params* p, int step, int v_begin, int v_count, const void* h_dev,
+                             const void* W_shard_dev, const void* E_shard_dev, const uint64_t* seeds_dev,
+                             void* partial_dev, void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/*
+ * Finish a step from the partials of n_parts shards that together cover the
+ * vocabulary once (1 <= n_parts <= 64; partials_dev holds them back to back):
+ * the merged entropy, argmax (smallest index on exact ties), log-sum-exp and
+ * self-conditioning vectors, the accept / re-noise of every position (or of the
+ * canvas's group, accept_rule 1) and the stop reduction - the outputs, state and
+ * arguments of dg_denoise_step.  Every device of a split runs the same merge on
+ * the same partials, so their canvases and stop flags stay identical.  A shard
+ * whose pass recorded an error poisons the merged results as described above.
+ */
+dg_status dg_denoise_merge(const dg_params* p, int step, int n_parts, const void* partials_dev,
+                           const uint64_t* seeds_dev, int32_t* tokens_dev, float* entropy_dev, int32_t* argmax_dev,
+                           uint8_t* accept_dev, float* lse_dev, float* selfcond_dev, void* workspace_dev,
+                           size_t workspace_bytes, void* stream);
 
 /* Column-slice group size and group count the fused kernel uses for p on the current device. */
 dg_status dg_plan(const dg_params* p, int* group, int* n_groups, int* slice_cols);

@@ -382,8 +382,8 @@ def stub_hidden(E_u16, tokens, seed, s, c, max_steps, gain=1.0, noise=0.1):
     n_{4j+2}, n_{4j+3}.  Computed in double, rounded to bf16 through float32.
     This stand-in is not on the pages; its realism is "parity unpinned".
     """
-    E = bf16_to_f64(E_u16)
-    V, d = E.shape
+    E_u16 = np.asarray(E_u16)
+    V, d = E_u16.shape
     tokens = np.asarray(tokens, np.int64)
     n = tokens.shape[0]
     a = s / max_steps
@@ -399,5 +399,6 @@ def stub_hidden(E_u16, tokens, seed, s, c, max_steps, gain=1.0, noise=0.1):
     nz = np.stack([ra * np.cos(2 * np.pi * u2a), ra * np.sin(2 * np.pi * u2a),
                    rb * np.cos(2 * np.pi * u2b), rb * np.sin(2 * np.pi * u2b)], axis=-1)
     nz = nz.reshape(n, d)
-    h = gain * (a * E[tgt] + (1.0 - a) * E[tokens]) + noise * nz
+    # only the gathered rows are widened (the values are those of the whole widened table)
+    h = gain * (a * bf16_to_f64(E_u16[tgt]) + (1.0 - a) * bf16_to_f64(E_u16[tokens])) + noise * nz
     return f64_to_bf16(h), tgt

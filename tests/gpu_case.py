@@ -20,6 +20,14 @@ H_TOL = 1e-3
 SC_TOL = 2e-2
 EXCL = 1e-3
 
+# (tag, rows compared, rows excluded) of every compare() in this session; printed by
+# tests/conftest.py at the end of the run
+REPORT = []
+
+
+def report(tag, n_rows, n_excluded, extra=""):
+    REPORT.append((tag, int(n_rows), int(n_excluded), extra))
+
 
 def to_dev(t):
     return t.to("cuda")
@@ -93,6 +101,7 @@ def compare(gpu, ora, rows, bound, check_selfcond=True, tag=""):
         rel = np.linalg.norm(a - b, axis=1) / np.maximum(np.linalg.norm(b, axis=1), 1e-30)
         esc = float(rel.max())
         assert esc <= SC_TOL, f"{tag}: self-conditioning rel L2 {esc:.3e} at row {rows[int(rel.argmax())]}"
+    report(tag, len(rows), int(np.count_nonzero(excl)), f"max|dH|={dH.max():.1e} sc={esc:.1e}")
     return rows[excl].tolist(), float(dH.max()), esc
 
 

@@ -36,3 +36,26 @@ def test_warmup_floor():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--warmup", "2"], capture_output=True,
                          text=True, timeout=120, cwd=ROOT)
     assert out.returncode != 0 and "warmup" in out.stderr
+
+
+def test_peak_follows_the_timed_regime():
+    """The roofline peak is the burst bf16 figure unless the timed region lasted a second or more
+    with the power cap active, where the sustained (seconds-long loop) figure applies."""
+    sys.path.insert(0, ROOT)
+    import bench
+    pk = {"bf16_tflops": 1644.9, "bf16_tflops_sustained": 1403.3}
+    assert bench.choose_peak(pk, 0.013, {"reasons": []}) == (1644.9, "burst")
+    assert bench.choose_peak(pk, 0.013, {"reasons": ["sw_power_cap"]}) == (1644.9, "burst")
+    assert bench.choose_peak(pk, 2.4, {"reasons": []}) == (1644.9, "burst")
+    assert bench.choose_peak(pk, 2.4, {"reasons": ["sw_power_cap"]}) == (1403.3, "sustained")
+
+
+def test_clock_summary_keeps_the_timed_window():
+    sys.path.insert(0, ROOT)
+    import bench
+    c = bench.ClockSampler(0)
+    c.max_mhz = 1965
+    c.rows = [(1.0, 1965, 300.0, 0x0), (2.0, 1900, 900.0, 0x4), (2.5, 1850, 950.0, 0x4), (4.0, 1000, 300.0, 0x8)]
+    s = c.summary(1.5, 3.0)
+    assert s["samples"] == 2 and s["sm_mhz"] == 1875 and s["reasons"] == ["sw_power_cap"] and s["sm_max_mhz"] == 1965
+    assert c.summary(5.0, 6.0)["reasons"] == ["no samples"]

@@ -12,7 +12,7 @@ import torch
 
 import gpu_case as gc
 import synth
-from oracle import philox, stage
+from oracle import decode, philox, stage
 
 pytestmark = pytest.mark.gpu
 
@@ -24,12 +24,6 @@ def dg():
     import discrete_diffusion_decoding_b200 as m
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     return m
-
-
-@pytest.fixture(scope="module")
-def big_W():
-    W = synth.weights(262144, 2816, seed=1234)
-    return W, gc.bits(W), W.cuda()
 
 
 def _assert_stub_close(got_bits, want_bits, gain):
@@ -153,45 +147,6 @@ def test_uniform_logits_closed_form(dg):
     assert rel.max() < 1e-3
 
 
-# ------------------------------------------------------------------ full-size single step
-def _sample_rows(N, n, seed):
-    rng = np.random.default_rng(seed)
-    fixed = [0, 1, 127, 128, 255, N - 1]
-    return np.unique(np.concatenate([fixed, rng.choice(N, size=n, replace=False)]))
-
-
-@pytest.mark.parametrize("hidden_kind,step,S", [("gaussian", 1, 48), ("spiked", 48, 48)])
-def test_full_vocab_single_step(dg, big_W, hidden_kind, step, S):
-    W, Wb, Wd = big_W
-    V, d, C = 262144, 2816, 1
-    if hidden_kind == "gaussian":
-        h = synth.gaussian_hidden(256, d, seed=42)
-    else:
-        h, _ = synth.spiked_hidden(W, 256, seed=43, gain_lo=2.0, gain_hi=40.0)
-    p = dg.params(C, V, d, max_steps=S)
-    seeds = synth.canvas_seeds(C)
-    g = gc.gpu_step(dg, p, step, h, Wd, Wd, seeds)
-    rows = _sample_rows(256, 40, 1)
-    o = gc.oracle_rows(gc.bits(h), Wb, Wb, dg.temperature(p, step), p.eb_bound, seeds, step, rows, V)
-    gc.compare(g, o, rows, p.eb_bound, tag=hidden_kind)
-    # properties that hold at every position
-    assert np.all(g["H"] >= -1e-4) and np.all(g["H"] <= math.log(V) + 1e-3)
-    assert np.all((g["argmax"] >= 0) & (g["argmax"] < V))
-
-
-def test_batched_full_vocab_step(dg, big_W):
-    """16 canvases (N = 4096) in one launch, per-canvas seeds: sampled rows in every canvas."""
-    W, Wb, Wd = big_W
-    V, d, C = 262144, 2816, 16
-    h, _ = synth.spiked_hidden(W, C * 256, seed=60, gain_lo=2.0, gain_hi=40.0)
-    p = dg.params(C, V, d)
-    seeds = synth.canvas_seeds(C, base=1000)
-    g = gc.gpu_step(dg, p, 7, h, Wd, Wd, seeds)
-    rows = _sample_rows(C * 256, 48, 2)
-    o = gc.oracle_rows(gc.bits(h), Wb, Wb, dg.temperature(p, 7), p.eb_bound, seeds, 7, rows, V)
-    gc.compare(g, o, rows, p.eb_bound, tag="batched")
-
-
 # ------------------------------------------------------------------ multi-step, lock-step
 def _lockstep(dg, V, d, C, S, gain, noise, seeds, W, sample=None, expect_stop=True):
     p = dg.params(C, V, d, max_steps=S)
@@ -263,10 +218,69 @@ def test_lockstep_batched_per_canvas_stop(dg):
 
 
 def test_lockstep_literal_gain_never_accepts(dg):
-    """The literal small configuration (gain 1): entropies stay near ln V, nothing is accepted."""
+    """The literal small configuration (gain 1, 16-step schedule, all 16 steps): entropies stay near
+    ln V, nothing is accepted, no stop; every position of every step against the oracle."""
     W = synth.weights(4096, 128)
-    stop_at = _lockstep(dg, 4096, 128, 1, 4, 1.0, 0.1, synth.canvas_seeds(1), W, expect_stop=False)
-    assert stop_at == [4]
+    stop_at = _lockstep(dg, 4096, 128, 1, 16, 1.0, 0.1, synth.canvas_seeds(1), W, expect_stop=False)
+    assert stop_at == [16]
+
+
+# ------------------------------------------------------------------ the product's decode loops
+def _record_steps(dg):
+    rec = {}
+
+    def on_step(s, bufs):
+        rec[s] = {"h": gc.bits(bufs.h).copy(), "tokens": bufs.tokens.cpu().numpy().astype(np.int64),
+                  "argmax": bufs.argmax.cpu().numpy().astype(np.int64)}
+    return rec, on_step
+
+
+def _oracle_replay(Wb, seeds, V, S, rec, canvas_ids, C):
+    """oracle.decode.decode_batch fed, at every step, the hidden states the GPU's stub produced for
+    that step (lock-step) - after checking that the oracle's canvas equals the one the GPU stub read."""
+    def hidden(tok, s, c):
+        want_in = rec[s - 1]["tokens"][c * 256:(c + 1) * 256] if s > 1 else tok
+        assert np.array_equal(tok, want_in), f"canvas {c} diverged before step {s}"
+        return rec[s]["h"][c * 256:(c + 1) * 256]
+    return decode.decode_batch(Wb, Wb, seeds, hidden, V, max_steps=S, record=True)
+
+
+def test_product_decode_batch_matches_oracle(dg):
+    """dg.decode_batch itself (stub inside, dg_stop_check every step, committed = the argmax of each
+    canvas's last step) against oracle.decode.decode_batch in lock-step on the GPU stub's h."""
+    V, d, C, S = 4096, 128, 3, 16
+    W = synth.weights(V, d)
+    Wb, Wd = gc.bits(W), W.cuda()
+    p = dg.params(C, V, d, max_steps=S)
+    seeds = synth.canvas_seeds(C, base=30)
+    seeds_t = torch.tensor(seeds.view(np.int64), device="cuda")
+    rec, on_step = _record_steps(dg)
+    committed, stop_step = dg.decode_batch(p, Wd, Wd, seeds_t, gain=300.0, noise=0.1, on_step=on_step)
+    ora = _oracle_replay(Wb, seeds, V, S, rec, None, C)
+    assert list(ora["stop_step"]) == list(stop_step)
+    assert min(stop_step) < S
+    assert np.array_equal(committed.cpu().numpy(), ora["committed"])
+    gc.report("decode_batch product loop", C * 256, 0, f"stop steps {stop_step}")
+
+
+def test_product_decode_block_ar_matches_oracle(dg):
+    """dg.decode_block_ar: 3 blocks one after another (seeds 7, 8, 9), each against the oracle's decode."""
+    V, d, S, n_blocks = 4096, 128, 16, 3
+    W = synth.weights(V, d)
+    Wb, Wd = gc.bits(W), W.cuda()
+    p1 = dg.params(1, V, d, max_steps=S)
+    recs = {}
+
+    def on_step(b, s, bufs):
+        recs.setdefault(b, {})[s] = {"h": gc.bits(bufs.h).copy(),
+                                     "tokens": bufs.tokens.cpu().numpy().astype(np.int64)}
+    out, steps = dg.decode_block_ar(p1, Wd, Wd, n_blocks, seed0=7, gain=300.0, noise=0.1, on_step=on_step)
+    out = out.cpu().numpy()
+    for b in range(n_blocks):
+        ora = _oracle_replay(Wb, np.array([7 + b], np.uint64), V, S, recs[b], None, 1)
+        assert int(ora["stop_step"][0]) == steps[b]
+        assert np.array_equal(out[b * 256:(b + 1) * 256], ora["committed"][0])
+    gc.report("decode_block_ar product loop", n_blocks * 256, 0, f"stop steps {steps}")
 
 
 # ------------------------------------------------------------------ argument checks
@@ -295,16 +309,39 @@ def test_argument_errors(dg):
         dg.dg_denoise_step(p, 1, bufs.h, W, W, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept, None,
                            None, small)
     assert e.value.status == _abi.DG_ENOMEM
-    with pytest.raises(_abi.DgError):
-        dg.workspace_size(dg.params(1, 4000, 128))            # vocab not a multiple of 256
-    with pytest.raises(_abi.DgError):
-        dg.workspace_size(dg.params(1, 4096, 100))            # hidden not a multiple of 64
-    with pytest.raises(_abi.DgError):
-        dg.workspace_size(dg.params(1, 4096, 192))            # no column slice of 128 or 256 divides it
-    bad = dg.params(1, 4096, 512, group=3)
-    with pytest.raises(_abi.DgError) as e:
-        dg.plan(bad)
-    assert e.value.status == _abi.DG_EUNSUPPORTED
+    # every limit the header states for dg_params, with the status it names
+    einval = [dict(n_canvas=0), dict(n_canvas=257), dict(canvas_len=128), dict(vocab=4000), dict(vocab=0),
+              dict(hidden=100), dict(hidden=64), dict(hidden=192), dict(max_steps=0), dict(t_start=0.0),
+              dict(t_end=-0.4), dict(stability=-1), dict(accept_mode=2), dict(accept_rule=-1)]
+    for bad in einval:
+        q = dg.params(1, 4096, 128)
+        for k, v in bad.items():
+            setattr(q, k, v)
+        with pytest.raises(_abi.DgError) as e:
+            dg.plan(q)
+        assert e.value.status == _abi.DG_EINVAL, bad
+        with pytest.raises(_abi.DgError):
+            dg.workspace_size(q)
+    eunsup = [(512, 3),        # the group does not divide hidden
+              (384, 2),        # slice 192: not a multiple of 128
+              (1280, 2),       # slice 640: wider than 256
+              (128 * 75, 75)]  # 75 pairs of CTAs: more than a B200 holds at once
+    for hidden, group in eunsup:
+        with pytest.raises(_abi.DgError) as e:
+            dg.plan(dg.params(1, 4096, hidden, group=group))
+        assert e.value.status == _abi.DG_EUNSUPPORTED, (hidden, group)
+    assert dg.plan(dg.params(256, 256, 128))["slice"] == 128       # the smallest accepted shape
+    # the vocabulary split's arguments
+    part = torch.empty(dg.dg_partial_bytes(p), dtype=torch.uint8, device="cuda")
+    for vb, vc in [(128, 256), (0, 0), (0, 300), (3840, 512), (-256, 512)]:
+        with pytest.raises(_abi.DgError) as e:
+            dg.dg_denoise_partial(p, 1, vb, vc, bufs.h, W, W, seeds, part, ws)
+        assert e.value.status == _abi.DG_EINVAL, (vb, vc)
+    for n_parts in (0, 65):
+        with pytest.raises(_abi.DgError) as e:
+            dg.dg_denoise_merge(p, 1, n_parts, part, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept,
+                                None, None, ws)
+        assert e.value.status == _abi.DG_EINVAL
     assert dg.last_launch_count() == 0
 
 
@@ -321,10 +358,17 @@ def test_forced_error_word_reported_and_cleared(dg):
     bufs.h.copy_(synth.gaussian_hidden(256, d).cuda())
     assert dg.dg_stop_check(p, ws)[2] == 0
     dg.dg_debug_set_error(p, ws, 301)
-    dg.dg_denoise_step(p, 1, bufs.h, W, W, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept, None, None, ws)
+    dg.dg_denoise_step(p, 1, bufs.h, W, W, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept, bufs.lse,
+                       bufs.selfcond, ws)
     with pytest.raises(_abi.DgError) as e:
         dg.dg_stop_check(p, ws)
     assert e.value.status == _abi.DG_ETIMEOUT
+    # the step's results are poisoned, not plausible: NaN entropy / LSE / self-conditioning,
+    # argmax -1, nothing accepted, every position re-noised (tokens stay in range)
+    assert torch.isnan(bufs.entropy).all() and torch.isnan(bufs.lse).all() and torch.isnan(bufs.selfcond).all()
+    assert (bufs.argmax == -1).all() and int(bufs.accept.sum()) == 0
+    want = stage.renoise_tokens(0, 1, 0, V)
+    assert np.array_equal(bufs.tokens.cpu().numpy(), want)
     with pytest.raises(_abi.DgError) as e:                 # the word stays set until the canvas is re-initialised
         dg.dg_stop_check(p, ws)
     assert e.value.status == _abi.DG_ETIMEOUT
@@ -369,7 +413,7 @@ def test_all_canvases_stopped_step_is_a_no_op(dg):
 
 
 def test_maximum_canvases_per_launch(dg):
-    """256 canvases (N = 65536) in one launch: sampled rows of many canvases against the oracle; 257 is refused."""
+    """256 canvases (N = 65536) in one launch: every position against the oracle; 257 is refused."""
     from discrete_diffusion_decoding_b200 import _abi
     V, d, C = 4096, 128, 256
     W = synth.weights(V, d)
@@ -378,8 +422,7 @@ def test_maximum_canvases_per_launch(dg):
     seeds = synth.canvas_seeds(C, base=500)
     Wd = W.cuda()
     g = gc.gpu_step(dg, p, 2, h, Wd, Wd, seeds)
-    rng = np.random.default_rng(12)
-    rows = np.unique(np.concatenate([[0, 255, 256, C * 256 - 1], rng.choice(C * 256, 60, replace=False)]))
+    rows = _rows_all(C * 256)
     o = gc.oracle_rows(gc.bits(h), gc.bits(W), gc.bits(W), dg.temperature(p, 2), p.eb_bound, seeds, 2, rows, V)
     gc.compare(g, o, rows, p.eb_bound, tag="256 canvases")
     assert np.all(g["stable"] == 0) and np.all(g["stop"] == 0)      # step 2 of a fresh run: nothing stable yet

@@ -1,0 +1,149 @@
+"""GPU parity of the vocabulary-parallel split: a head cut into vocabulary shards, each
+shard's fused pass writing a partial (dg_denoise_partial), the partials merged
+(dg_denoise_merge).  On one GPU the shards run one after another into one buffer, as
+the all-gather of a multi-GPU split would lay them out.
+
+The merged results equal the single call's (the logits of a row are the same numbers
+whatever the split, so argmax, accept flags and tokens are identical; entropy and
+self-conditioning agree to rounding) and the oracle's under the usual tolerances.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import gpu_case as gc
+import synth
+from oracle import stage
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dg():
+    from discrete_diffusion_decoding_b200 import build
+    build.build()
+    import discrete_diffusion_decoding_b200 as m
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return m
+
+
+def _split_step(dg, p, step, h, W, E, seeds_t, bounds, tokens_in, ws=None, bufs=None, prepare=None):
+    """One step through partial + merge over the given shard bounds; returns host outputs."""
+    ws = ws or dg.Workspace(p)
+    bufs = bufs or dg.StepBuffers(p)
+    nb = dg.dg_partial_bytes(p)
+    parts = torch.empty(len(bounds) * nb, dtype=torch.uint8, device="cuda")
+    if tokens_in is not None:
+        dg.dg_canvas_init(p, seeds_t, bufs.tokens, ws)
+        bufs.tokens.copy_(torch.as_tensor(np.asarray(tokens_in, np.int32)).cuda())
+    bufs.h.copy_(h.cuda() if not h.is_cuda else h)
+    for k, (v0, v1) in enumerate(bounds):
+        if prepare is not None:
+            prepare(k)
+        dg.dg_denoise_partial(p, step, v0, v1 - v0, bufs.h, W[v0:v1], E[v0:v1], seeds_t, parts[k * nb:(k + 1) * nb],
+                              ws)
+        assert dg.last_launch_count() == 2
+    dg.dg_denoise_merge(p, step, len(bounds), parts, seeds_t, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept,
+                        bufs.lse, bufs.selfcond, ws)
+    assert dg.last_launch_count() == 2
+    flags, stable, _ = dg.dg_stop_check(p, ws, want_stable=True)
+    return {"H": bufs.entropy.cpu().numpy().astype(np.float64), "argmax": bufs.argmax.cpu().numpy().astype(np.int64),
+            "tokens": bufs.tokens.cpu().numpy().astype(np.int64), "accept": bufs.accept.cpu().numpy(),
+            "lse": bufs.lse.cpu().numpy().astype(np.float64),
+            "selfcond": bufs.selfcond.cpu().numpy().astype(np.float64), "stop": np.array(flags),
+            "stable": np.array(stable)}
+
+
+@pytest.mark.parametrize("V,d,C,group,bounds,tied,mode,rule,bound", [
+    (8960, 512, 2, 2, [(0, 4608), (4608, 8960)], True, 0, 0, 0.1),
+    (8960, 512, 2, 4, [(0, 256), (256, 6144), (6144, 8960)], False, 0, 0, 0.1),
+    (4096, 128, 3, 0, [(0, 1024), (1024, 2048), (2048, 3072), (3072, 4096)], True, 1, 0, 6.0),
+    (4096, 128, 3, 0, [(0, 2048), (2048, 4096)], True, 0, 1, 2.0),
+])
+def test_shards_merge_to_single_call_and_oracle(dg, V, d, C, group, bounds, tied, mode, rule, bound):
+    W = synth.weights(V, d, seed=1234)
+    E = W if tied else synth.weights(V, d, seed=1235)
+    h, _ = synth.spiked_hidden(W, C * 256, seed=90 + len(bounds), gain_lo=0.5, gain_hi=30.0)
+    p = dg.params(C, V, d, group=group, tied=int(tied), accept_mode=mode, accept_rule=rule, eb_bound=bound)
+    seeds = synth.canvas_seeds(C, base=400)
+    seeds_t = torch.tensor(seeds.view(np.int64), device="cuda")
+    Wd = W.cuda()
+    Ed = Wd if tied else E.cuda()
+    step = 5
+    single = gc.gpu_step(dg, p, step, h, Wd, Ed, seeds)
+    tok0 = np.concatenate([stage.init_tokens(int(seeds[c]), c, V) for c in range(C)])
+    split = _split_step(dg, p, step, h, Wd, Ed, seeds_t, bounds, tok0)
+    # the same logits whatever the split: identical decisions, entropies and vectors to rounding
+    assert np.array_equal(split["argmax"], single["argmax"])
+    assert np.abs(split["H"] - single["H"]).max() <= 1e-4
+    near = np.abs(single["H"] - bound) < 1e-4
+    assert np.array_equal(split["accept"][~near], single["accept"][~near]) or rule == 1
+    rel = np.linalg.norm(split["selfcond"] - single["selfcond"], axis=1) / np.linalg.norm(single["selfcond"], axis=1)
+    assert rel.max() <= 1e-4
+    rows = np.arange(C * 256)
+    T = dg.temperature(p, step)
+    if rule == 0:
+        o = gc.oracle_rows(gc.bits(h), gc.bits(W), gc.bits(E), T, bound, seeds, step, rows, V, accept_mode=mode)
+        gc.compare(split, o, rows, bound, tag=f"vocab split {len(bounds)} shards mode={mode}")
+    else:
+        o = gc.oracle_rows(gc.bits(h), gc.bits(W), gc.bits(E), T, bound, seeds, step, rows, V, want_selfcond=False)
+        assert np.abs(split["H"] - o["H"]).max() <= gc.H_TOL
+        assert np.array_equal(split["accept"], single["accept"]) and np.array_equal(split["tokens"], single["tokens"])
+        gc.report(f"vocab split group rule {len(bounds)} shards", C * 256, 0, "accept/tokens = single call")
+        assert 0 < int(split["accept"].sum()) < C * 256
+
+
+def test_split_lockstep_decode_with_stops(dg):
+    """A stub-driven decode of 2 canvases where every step runs as two shards + merge: every position
+    against the oracle each step; canvases stop (stopped ones are skipped by both halves)."""
+    V, d, C, S, gain = 4096, 128, 2, 16, 300.0
+    W = synth.weights(V, d)
+    Wb, Wd = gc.bits(W), W.cuda()
+    p = dg.params(C, V, d, max_steps=S)
+    ws, bufs = dg.Workspace(p), dg.StepBuffers(p)
+    seeds = synth.canvas_seeds(C, base=80)
+    seeds_t = torch.tensor(seeds.view(np.int64), device="cuda")
+    dg.dg_canvas_init(p, seeds_t, bufs.tokens, ws)
+    bounds = [(0, 1536), (1536, 4096)]
+    stopped = [False] * C
+    stop_at = [S] * C
+    for s in range(1, S + 1):
+        tok_in = bufs.tokens.cpu().numpy().copy()
+        dg.dg_stub_hidden(p, s, gain, 0.1, seeds_t, Wd, bufs.tokens, bufs.h, ws)
+        hb = gc.bits(bufs.h)
+        g = _split_step(dg, p, s, bufs.h, Wd, Wd, seeds_t, bounds, None, ws=ws, bufs=bufs)
+        for c in range(C):
+            sl = slice(c * 256, (c + 1) * 256)
+            if stopped[c]:
+                assert np.array_equal(g["tokens"][sl], tok_in[sl])
+                continue
+            rows = np.arange(c * 256, (c + 1) * 256)
+            o = gc.oracle_rows(hb, Wb, Wb, dg.temperature(p, s), p.eb_bound, seeds, s, rows, V)
+            gc.compare(g, o, rows, p.eb_bound, tag=f"split decode s={s} c={c}")
+            if g["stop"][c]:
+                stopped[c] = True
+                stop_at[c] = s
+        if all(stopped):
+            break
+    assert min(stop_at) < S and min(stop_at) >= 3
+
+
+def test_poisoned_shard_poisons_the_merge(dg):
+    """A shard whose pass recorded an error (injected on the host into its workspace's error word)
+    makes every merged position NaN / -1, not a plausible result from the other shard alone."""
+    V, d, C = 4096, 128, 1
+    W = synth.weights(V, d)
+    Wd = W.cuda()
+    p = dg.params(C, V, d)
+    ws = dg.Workspace(p)
+    seeds_t = torch.zeros(1, dtype=torch.int64, device="cuda")
+    h = synth.gaussian_hidden(256, d)
+    tok0 = stage.init_tokens(0, 0, V)
+
+    def prepare(k):
+        if k == 1:
+            dg.dg_debug_set_error(p, ws, 302)
+    out = _split_step(dg, p, 1, h, Wd, Wd, seeds_t, [(0, 2048), (2048, 4096)], tok0, ws=ws, prepare=prepare)
+    assert np.isnan(out["H"]).all() and np.isnan(out["selfcond"]).all() and np.all(out["argmax"] == -1)
+    assert int(out["accept"].sum()) == 0 and out["tokens"].min() >= 0 and out["tokens"].max() < V

@@ -32,36 +32,39 @@ def dg():
     return m
 
 
-def _regular(dg, p, step, h, W):
+def _regular(dg, p, step, h, W, E):
     ws = dg.Workspace(p)
     b = dg.StepBuffers(p)
     seeds = torch.zeros(p.n_canvas, dtype=torch.int64, device="cuda")
     dg.dg_canvas_init(p, seeds, b.tokens, ws)
     b.h.copy_(h)
-    dg.dg_denoise_step(p, step, b.h, W, W, seeds, b.tokens, b.entropy, b.argmax, b.accept, b.lse, b.selfcond, ws)
+    dg.dg_denoise_step(p, step, b.h, W, E, seeds, b.tokens, b.entropy, b.argmax, b.accept, b.lse, b.selfcond, ws)
     dg.dg_stop_check(p, ws)
     return b.entropy.clone(), b.argmax.clone(), b.lse.clone(), b.selfcond.clone()
 
 
-def test_noalloc_matches_workspace_path_on_two_calls(dg):
+@pytest.mark.parametrize("tied", [True, False])
+def test_noalloc_matches_workspace_path_on_two_calls(dg, tied):
     V, d, C = 32768, 2816, 2
     W = synth.weights(V, d).cuda()
+    E = W if tied else synth.weights(V, d, seed=1235).cuda()
     h, _ = synth.spiked_hidden(W.cpu(), C * 256, seed=77, gain_lo=1.0, gain_hi=40.0)
     h = h.cuda()
-    p = dg.params(C, V, d)
+    p = dg.params(C, V, d, tied=int(tied))
     N = C * 256
     H = torch.empty(N, dtype=torch.float32, device="cuda")
     am = torch.empty(N, dtype=torch.int32, device="cuda")
     lse = torch.empty(N, dtype=torch.float32, device="cuda")
     sc = torch.empty((N, d), dtype=torch.float32, device="cuda")
     for call, step in enumerate((1, 48)):
-        want = _regular(dg, p, step, h, W)
+        want = _regular(dg, p, step, h, W, E)
         torch.cuda.synchronize()
         free_before = torch.cuda.mem_get_info()[0]
         H.fill_(float("nan"))
         am.fill_(-7)
         sc.fill_(float("nan"))
-        dg.dg_denoise_stats_noalloc(p, step, h, W, W, H, am, lse, sc)
+        dg.dg_denoise_stats_noalloc(p, step, h, W, E, H, am, lse, sc)
+        assert dg.last_launch_count() == 3            # clear, fused pass, combine
         torch.cuda.synchronize()
         if call > 0:
             # the first call on a device is its set-up (the runtime may load the
@@ -79,6 +82,13 @@ def test_noalloc_matches_workspace_path_on_two_calls(dg):
 def test_noalloc_refuses_shapes_beyond_its_scratch(dg):
     from discrete_diffusion_decoding_b200 import _abi
     V, d = 262144, 2816
+    # the documented limit: up to 4 canvases of this head fit the 64 MiB scratch, 5 do not
+    assert dg.workspace_size(dg.params(4, V, d)) <= 64 << 20 < dg.workspace_size(dg.params(5, V, d))
+    x = torch.empty(16, dtype=torch.float32, device="cuda")
+    with pytest.raises(_abi.DgError) as e:
+        dg.dg_denoise_stats_noalloc(dg.params(5, V, d), 1, x, x, x, x, x, None, None)
+    assert e.value.status == _abi.DG_ENOMEM
+    assert dg.last_launch_count() == 0
     p = dg.params(64, V, d)                    # needs far more than the fixed scratch
     x = torch.empty(16, dtype=torch.float32, device="cuda")
     with pytest.raises(_abi.DgError) as e:
