@@ -79,8 +79,10 @@ def test_shards_merge_to_single_call_and_oracle(dg, V, d, C, group, bounds, tied
     assert np.abs(split["H"] - single["H"]).max() <= 1e-4
     near = np.abs(single["H"] - bound) < 1e-4
     assert np.array_equal(split["accept"][~near], single["accept"][~near]) or rule == 1
+    # P is rounded to bf16 against a reference maximum that depends on which rows a group streams,
+    # so the vectors differ at the level of that rounding (the oracle bound below is the contract)
     rel = np.linalg.norm(split["selfcond"] - single["selfcond"], axis=1) / np.linalg.norm(single["selfcond"], axis=1)
-    assert rel.max() <= 1e-4
+    assert rel.max() <= gc.SC_TOL
     rows = np.arange(C * 256)
     T = dg.temperature(p, step)
     if rule == 0:
