@@ -28,7 +28,8 @@ def dg():
     return m
 
 
-def _split_step(dg, p, step, h, W, E, seeds_t, bounds, tokens_in, ws=None, bufs=None, prepare=None):
+def _split_step(dg, p, step, h, W, E, seeds_t, bounds, tokens_in, ws=None, bufs=None, prepare=None,
+                expect_timeout=False):
     """One step through partial + merge over the given shard bounds; returns host outputs."""
     ws = ws or dg.Workspace(p)
     bufs = bufs or dg.StepBuffers(p)
@@ -47,7 +48,14 @@ def _split_step(dg, p, step, h, W, E, seeds_t, bounds, tokens_in, ws=None, bufs=
     dg.dg_denoise_merge(p, step, len(bounds), parts, seeds_t, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept,
                         bufs.lse, bufs.selfcond, ws)
     assert dg.last_launch_count() == 2
-    flags, stable, _ = dg.dg_stop_check(p, ws, want_stable=True)
+    if expect_timeout:
+        from discrete_diffusion_decoding_b200 import _abi
+        with pytest.raises(_abi.DgError) as e:
+            dg.dg_stop_check(p, ws)
+        assert e.value.status == _abi.DG_ETIMEOUT
+        flags = stable = [0] * p.n_canvas
+    else:
+        flags, stable, _ = dg.dg_stop_check(p, ws, want_stable=True)
     return {"H": bufs.entropy.cpu().numpy().astype(np.float64), "argmax": bufs.argmax.cpu().numpy().astype(np.int64),
             "tokens": bufs.tokens.cpu().numpy().astype(np.int64), "accept": bufs.accept.cpu().numpy(),
             "lse": bufs.lse.cpu().numpy().astype(np.float64),
@@ -146,6 +154,7 @@ def test_poisoned_shard_poisons_the_merge(dg):
     def prepare(k):
         if k == 1:
             dg.dg_debug_set_error(p, ws, 302)
-    out = _split_step(dg, p, 1, h, Wd, Wd, seeds_t, [(0, 2048), (2048, 4096)], tok0, ws=ws, prepare=prepare)
+    out = _split_step(dg, p, 1, h, Wd, Wd, seeds_t, [(0, 2048), (2048, 4096)], tok0, ws=ws, prepare=prepare,
+                      expect_timeout=True)
     assert np.isnan(out["H"]).all() and np.isnan(out["selfcond"]).all() and np.all(out["argmax"] == -1)
     assert int(out["accept"].sum()) == 0 and out["tokens"].min() >= 0 and out["tokens"].max() < V
