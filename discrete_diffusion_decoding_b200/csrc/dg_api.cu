@@ -176,9 +176,8 @@ dg_status make_plan(const dg_params* p, int pairs, Plan* pl) {
     q.d = p->hidden;
     q.group = G;
     q.slice = slice;
-    q.pairs = pairs;
     q.n_groups = pairs / G;
-    q.steps_per_tile = (p->vocab + G * kBS - 1) / (G * kBS);
+    q.steps_per_tile = (p->vocab + G * kBV - 1) / (G * kBV);
     // partial slots per group: the most pieces any active-canvas count can give a group
     q.max_seg = 1;
     for (int n_ct = 1; n_ct <= q.C; ++n_ct) {
@@ -221,9 +220,9 @@ dg_status launch_fused_and_combine(const dg_params* p, const Plan& pl, const Lay
     const float T = dg_temperature(p, step);
     FusedArgs fa;
     std::memset(&fa, 0, sizeof(fa));
-    const uint64_t prow_total = static_cast<uint64_t>(pl.n_groups) * 2 * pl.group * kBS;   // P^T rows
+    const uint64_t prow_total = static_cast<uint64_t>(pl.n_groups) * 2 * pl.group * kCanvas;
     if (!encode_blocks_3d(&fa.map_h, io.h, pl.N, pl.d, kTileM, kKChunk / 64) ||
-        !encode_blocks_3d(&fa.map_w, io.W, io.vocab_rows, pl.d, kBS / 2, kKChunk / 64) ||
+        !encode_blocks_3d(&fa.map_w, io.W, io.vocab_rows, pl.d, kBV / 2, kKChunk / 64) ||
         !encode_blocks_3d(&fa.map_e, io.E, io.vocab_rows, pl.d, kVChunk, pl.slice / 128) ||
         !encode_blocks_3d(&fa.map_p, at<void>(ws, L.pbuf), prow_total, kCanvas, kVChunk, 2))
         return DG_ECUDA;
@@ -248,15 +247,13 @@ dg_status launch_fused_and_combine(const dg_params* p, const Plan& pl, const Lay
     fa.keep_w_stages = io.E == io.W ? (pl.d / kKChunk) * kKeepWTenths / 10 : 0;
     fa.slice = pl.slice;
     fa.n_groups = pl.n_groups;
-    fa.n_pairs = pl.pairs;
-    fa.placement = kPlacement;
-    fa.steps_per_tile = (io.vocab_rows + pl.group * kBS - 1) / (pl.group * kBS);
+    fa.steps_per_tile = (io.vocab_rows + pl.group * kBV - 1) / (pl.group * kBV);
     fa.max_seg = pl.max_seg;
     fa.scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
 
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(2 * pl.pairs);   // every resident pair: the placement needs all of them
+    cfg.gridDim = dim3(2 * pl.n_groups * pl.group);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kFusedSmem;
     cfg.stream = s;
@@ -414,7 +411,7 @@ dg_status dg_canvas_init(const dg_params* p, const uint64_t* seeds_dev, int32_t*
     dg_init_kernel<<<blocks, threads, 0, s>>>(seeds_dev, tokens_dev, at<int32_t>(workspace_dev, L.prev_argmax),
                                               at<int32_t>(workspace_dev, L.stable), at<int32_t>(workspace_dev, L.stop),
                                               at<int32_t>(workspace_dev, L.err), at<uint32_t>(workspace_dev, L.counters),
-                                              counter_words(pl.n_groups), pl.C, pl.V);
+                                              pl.n_groups * 128, pl.C, pl.V);
     if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
     g_last_launches = 1;
     return DG_OK;

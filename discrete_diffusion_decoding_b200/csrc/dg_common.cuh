@@ -12,8 +12,7 @@ namespace dg {
 
 constexpr int kCanvas = 256;      // positions per canvas
 constexpr int kTileM = 128;       // positions per tile (UMMA M)
-constexpr int kBV = 256;          // vocabulary granularity of the interface (shards, vocabulary size)
-constexpr int kBS = 128;          // vocabulary rows of one pair's logits sub-tile (UMMA N of the logits GEMM)
+constexpr int kBV = 256;          // vocabulary rows per logits tile (UMMA N)
 constexpr int kKChunk = 128;      // hidden columns per pipeline stage of the logits GEMM
 constexpr int kVChunk = 128;      // vocabulary rows per pipeline stage of the self-conditioning GEMM
 constexpr int kMaxSlice = 256;    // widest self-conditioning column slice a CTA pair keeps in TMEM
@@ -28,15 +27,21 @@ constexpr int kFusedStageBytes = 64 * 1024;
 #define DG_KEEP_W_TENTHS 3
 #endif
 constexpr int kKeepWTenths = DG_KEEP_W_TENTHS;
+// L2 prefetch distances of the fused kernel's streamed operands, in pipeline loads: the W
+// box this many loads ahead in the logits stream, and the E box this many loads ahead in
+// the self-conditioning stream, are requested into L2 when a load is issued, so that the
+// loads themselves find their bytes on chip (the three shared-memory stages alone cannot
+// cover DRAM latency at the full SM clock).
+#ifndef DG_PREFETCH_W
+#define DG_PREFETCH_W 8
+#endif
+#ifndef DG_PREFETCH_E
+#define DG_PREFETCH_E 8
+#endif
+constexpr int kPrefetchW = DG_PREFETCH_W;
+constexpr int kPrefetchE = DG_PREFETCH_E;
 constexpr int kFusedSmemBytes = kFusedStages * kFusedStageBytes + 1024 + 4 * kMaxCanvas;
 constexpr float kLazyRescale = 8.0f;  // log2 units the shared reference may lag the running max
-// How the fused kernel deals (group, sub-tile) roles to its CTA pairs: 0 by cluster index, 1 every
-// group within one half of the SM ids (one die of a two-die B200: a group's E re-reads of the W
-// rows its own pairs streamed then hit that die's L2).
-#ifndef DG_PLACEMENT
-#define DG_PLACEMENT 1
-#endif
-constexpr int kPlacement = DG_PLACEMENT;
 
 // ------------------------------------------------------------------ Philox4x32-10
 // Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3" (SC'11):
@@ -79,18 +84,17 @@ struct Plan {
     int C, N, V, d;
     int group;        // G: CTA pairs sharing one logits tile stream, each pair owning d/G columns
     int slice;        // d / G
-    int pairs;        // CTA pairs resident at once: the grid (pairs beyond n_groups * G idle)
-    int n_groups;     // groups of G pairs working at once
-    int steps_per_tile;  // vocabulary blocks of G * kBS rows per canvas
+    int n_groups;     // groups resident at once (grid = n_groups * G pairs = 2 n_groups G CTAs)
+    int steps_per_tile;  // vocabulary blocks of G * kBV rows per canvas
     int max_seg;      // partial slots per group
     int n_slots;      // n_groups * max_seg
 };
 
 struct Layout {
     size_t prev_argmax, stable, stop, err;        // per-canvas state
-    size_t counters;                              // [n_groups + 1][4] uint32, 128 B apart (the last: placement)
+    size_t counters;                              // [n_groups][4] uint32, 128 B apart
     size_t rowmax;                                // [n_groups][2][G][256] float
-    size_t pbuf;                                  // [n_groups][2][G][kBS vocab][256 rows] bf16 (P^T)
+    size_t pbuf;                                  // [n_groups][2][G][kBV vocab][256 rows] bf16 (P^T)
     size_t stats;                                 // [n_slots][G][256] float4 {m, l, u, best}
     size_t stat_idx;                              // [n_slots][G][256] int32
     size_t skey;                                  // [n_slots][G][256] float: best Gumbel-max key (sampled mode)
@@ -114,9 +118,9 @@ inline Layout make_layout(const Plan& pl) {
     L.stable = take(sizeof(int32_t) * pl.C);
     L.stop = take(sizeof(int32_t) * pl.C);
     L.err = take(sizeof(int32_t) * 4);
-    L.counters = take(static_cast<size_t>(128) * 4 * (pl.n_groups + 1));
+    L.counters = take(static_cast<size_t>(128) * 4 * pl.n_groups);
     L.rowmax = take(sizeof(float) * pl.n_groups * 2 * pl.group * kCanvas);
-    L.pbuf = take(static_cast<size_t>(2) * pl.n_groups * 2 * pl.group * kCanvas * kBS);
+    L.pbuf = take(static_cast<size_t>(2) * pl.n_groups * 2 * pl.group * kCanvas * kBV);
     L.stats = take(sizeof(float) * 4 * static_cast<size_t>(pl.n_slots) * pl.group * kCanvas);
     L.stat_idx = take(sizeof(int32_t) * static_cast<size_t>(pl.n_slots) * pl.group * kCanvas);
     L.skey = take(sizeof(float) * static_cast<size_t>(pl.n_slots) * pl.group * kCanvas);
@@ -166,10 +170,8 @@ __host__ __device__ inline bool piece_of(int g, int j, int n_groups, int n_pt, i
     return te > tb;
 }
 
-// Offsets of the four per-group counters (uint32 words); counter block n_groups holds the
-// placement counters of the fused kernel's prologue.
+// Offsets of the four per-group counters (uint32 words).
 enum : int { kCntRowmax = 0, kCntP = 1, kCntUsed = 2 };
-__host__ __device__ inline int counter_words(int n_groups) { return (n_groups + 1) * 128; }
 __host__ __device__ inline size_t counter_word(int g, int which) { return static_cast<size_t>(g) * 128 + which * 32; }
 
 }  // namespace dg

@@ -55,13 +55,11 @@ namespace dg {
 namespace {
 
 constexpr int kStages = kFusedStages;
-constexpr int kStageBytes = kFusedStageBytes;   // per CTA: A operand 32 KB + B operand 32 KB (logits: 16 KB)
+constexpr int kStageBytes = kFusedStageBytes;   // per CTA: A operand 32 KB + B operand half 32 KB
 constexpr int kHalfB = 32 * 1024;
 constexpr uint32_t kAtomCol = 128u * 128u;     // bytes of one 64-column swizzle atom column of a 128-row box
-constexpr uint32_t kAtomColW = 128u * (kBS / 2);   // the same for this CTA's kBS / 2 W rows
-constexpr uint32_t kSStageBytes = 2u * kAtomCol + 2u * kAtomColW;   // one logits stage: h 32 KB + W 16 KB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemS = 0;             // two logits buffers: columns [0, kBS) and [kBS, 2 kBS)
+constexpr uint32_t kTmemS = 0;             // logits tile columns [0, 256)
 constexpr uint32_t kTmemO = 256;           // self-conditioning slice columns [256, 256 + slice)
 constexpr int kSoftmaxWarp0 = 4;
 constexpr int kMaxSlotsPerTile = 256;      // >= ranges per tile (at most the group count)
@@ -71,7 +69,6 @@ enum : int {
     kErrProducerEmpty = 101, kErrProducerP = 102, kErrProducerDrain = 103,
     kErrMmaFull = 201, kErrMmaSFree = 202, kErrMmaOReady = 203, kErrMmaDrain = 204,
     kErrSmaxSFull = 301, kErrSmaxRowmax = 302, kErrSmaxUsed = 303, kErrSmaxODone = 304,
-    kErrPlace = 401,
 };
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
@@ -181,7 +178,7 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
     int* active = reinterpret_cast<int*>(ring + kStages * kStageBytes);
 
     __shared__ uint64_t full_bar[kStages], empty_bar[kStages];
-    __shared__ uint64_t s_full[2], s_free[2], o_ready, o_done, drain_bar;
+    __shared__ uint64_t s_full, s_free, o_ready, o_done, drain_bar;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     __shared__ int n_active_s;
@@ -193,54 +190,24 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
     const int G = a.G;
     const uint32_t prank = cluster_ctarank();        // 0 = pair leader (issues the UMMAs)
     const bool leader = prank == 0;
-    __shared__ int s_role;                           // g * G + r of this pair, -1 when idle
+    const int pair = blockIdx.x >> 1;
+    const int g = pair / G;
+    const int r = pair % G;
+    const int d0 = r * a.slice;
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&full_bar[i], 1);      // leader: one expect_tx arrival per use, bytes of both CTAs
             mbar_init(&empty_bar[i], 1);     // one multicast commit per use
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&s_full[i], 1);        // logits buffer i holds a finished tile
-            mbar_init(&s_free[i], 2);        // leader: softmax of both CTAs done reading buffer i
-        }
+        mbar_init(&s_full, 1);
+        mbar_init(&s_free, 2);               // leader: softmax of both CTAs
         mbar_init(&o_ready, 2);              // leader: softmax of both CTAs
         mbar_init(&o_done, 1);
         mbar_init(&drain_bar, 1);
         fence_mbar_init_cluster();
         abort_flag = 0;
         rescale_any = 0;
-        if (leader) {
-            // Role of this pair (group g, sub-tile r).  Placement 1 forms every group from pairs of
-            // one half of the SM id space - one die of a two-die part, whose L2 is the one that
-            // the group's E re-reads of its own W rows can hit - by arrival order within the half
-            // (every pair of the grid is resident, so all of them arrive).  Placement 0 (and a
-            // half that holds too few pairs for its groups) deals roles by cluster index.
-            int role = static_cast<int>(blockIdx.x >> 1);
-            const int n_roles = a.n_groups * G;
-            if (a.placement == 1) {
-                uint32_t smid, nsmid;
-                asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-                asm volatile("mov.u32 %0, %%nsmid;" : "=r"(nsmid));
-                const int die = smid >= (nsmid >> 1) ? 1 : 0;
-                uint32_t* place = a.counters + counter_word(a.n_groups, 0);   // [0], [1]: per half; [2]: all
-                const int pos = static_cast<int>(atomicAdd(place + die, 1u));
-                red_release_add(place + 2, 1u);
-                if (wait_counter(place + 2, static_cast<uint32_t>(a.n_pairs), &abort_flag, a.err, kErrPlace)) {
-                    const int c0 = static_cast<int>(__ldcg(place + 0));
-                    const int c1 = static_cast<int>(__ldcg(place + 1));
-                    const int q0 = min(a.n_groups, c0 / G), q1 = a.n_groups - q0;
-                    if (q1 * G <= c1)
-                        role = die == 0 ? (pos < q0 * G ? pos : -1) : (pos < q1 * G ? q0 * G + pos : -1);
-                    else
-                        role = die == 0 ? pos : c0 + pos;
-                } else {
-                    role = -1;
-                }
-            }
-            if (role >= n_roles) role = -1;
-            s_role = role;     // the peer CTA reads it from here after the cluster barrier below
-        }
     }
     if (warp == 2) {
         // active canvases in increasing order
@@ -263,20 +230,10 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
     tc_fence_after();
 
     const uint32_t tmem = tmem_base;
-    int role;
-    if (leader) {
-        role = s_role;
-    } else {
-        // the leader's decision, read from its shared memory (both CTAs have passed the barrier)
-        asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(role) : "r"(smem_addr_in_rank(&s_role, 0)) : "memory");
-    }
-    const int g = role >= 0 ? role / G : 0;
-    const int r = role >= 0 ? role % G : 0;
-    const int d0 = r * a.slice;
     Schedule sch;
     sch.init(g, a.n_groups, n_active_s, a.steps_per_tile);
-    auto sub_valid = [&](int t, int q) { return static_cast<long long>(t * G + q) * kBS < a.V; };
-    auto vocab0 = [&](int t, int q) { return (t * G + q) * kBS; };
+    auto sub_valid = [&](int t, int q) { return static_cast<long long>(t * G + q) * kBV < a.V; };
+    auto vocab0 = [&](int t, int q) { return (t * G + q) * kBV; };
 
     uint32_t* cnt_rowmax = a.counters + counter_word(g, kCntRowmax);
     uint32_t* cnt_p = a.counters + counter_word(g, kCntP);
@@ -285,9 +242,7 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
     const uint32_t o_stage_bytes = 2u * kAtomCol + static_cast<uint32_t>(n_ech) * kAtomCol;   // P^T 2 x 16 KB + E
     const int nG2 = 2 * G;                           // CTAs per group
 
-    if (role < 0) {
-        // idle pair: no work, straight to the teardown
-    } else if (warp == 0 || warp == 3) {
+    if (warp == 0 || warp == 3) {
         // ===================================================== TMA producers (both CTAs)
         // Warp 0 issues the A operand of every stage (h rows, or the P^T columns of
         // this CTA's positions) and posts the stage's expected bytes on the leader's
@@ -314,6 +269,21 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 ++it;
                 return true;
             };
+            const int nkc = a.d / kKChunk;                 // logits stages per W tile
+            const int ne = 2 * G;                          // self-conditioning E loads per block (full blocks)
+            // B side: the E box of load n of block t's self-conditioning stream (n may run into block t + 1)
+            auto prefetch_e = [&](int t, int n, int te) {
+                if (kPrefetchE <= 0) return;
+                while (n >= ne) {
+                    n -= ne;
+                    ++t;
+                }
+                const int q = n >> 1, vc = n & 1;
+                if (t < te && sub_valid(t, q))
+                    tma_prefetch_l2_3d(&a.map_e, 0, vocab0(t, q) + vc * kVChunk,
+                                       (d0 + static_cast<int>(prank) * (a.slice / 2)) / 64);
+            };
+            int piece_te = 0;
             auto emit_o = [&](int k, int t) -> bool {
                 if (a_side) {
                     if (!wait_counter(cnt_p, static_cast<uint32_t>(nG2 * (k + 1)), &abort_flag, a.err, kErrProducerP))
@@ -323,8 +293,8 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 for (int q = 0; q < G; ++q) {
                     if (!sub_valid(t, q)) continue;
                     // P^T tile of (block k, sub-tile q): [256 vocab rows][256 canvas rows]
-                    const int prow = ((g * 2 + (k & 1)) * G + q) * kBS;
-                    for (int vc = 0; vc < kBS / kVChunk; ++vc) {
+                    const int prow = ((g * 2 + (k & 1)) * G + q) * kBV;
+                    for (int vc = 0; vc < kBV / kVChunk; ++vc) {
                         int slot;
                         if (!acquire(slot)) return false;
                         uint8_t* st = ring + slot * kStageBytes;
@@ -334,6 +304,7 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                             tma_load_3d_pair(st, &a.map_p, full_leader(slot), 0, prow + vc * kVChunk,
                                              static_cast<int>(prank) * 2);
                         } else {
+                            prefetch_e(t, q * 2 + vc + kPrefetchE, piece_te);
                             // this CTA's half of the column slice (n_ech atoms of 64 columns) in one 3-D box
                             tma_load_3d_pair_hint(st + kHalfB, &a.map_e, full_leader(slot), 0,
                                                   vocab0(t, q) + vc * kVChunk,
@@ -348,15 +319,25 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 int ct, tb, te;
                 if (!sch.seg(j, ct, tb, te)) continue;
                 const int row0 = active[ct] * kCanvas + static_cast<int>(prank) * kTileM;
+                piece_te = te;
                 for (int t = tb; t < te && ok; ++t, ++k) {
                     if (sub_valid(t, r)) {
-                        const int v0 = vocab0(t, r) + static_cast<int>(prank) * (kBS / 2);
-                        for (int kc = 0; kc < a.d / kKChunk; ++kc) {
+                        const int v0 = vocab0(t, r) + static_cast<int>(prank) * (kBV / 2);
+                        for (int kc = 0; kc < nkc; ++kc) {
+                            if (!a_side && kPrefetchW > 0) {
+                                // the W box kPrefetchW loads ahead in this piece's logits stream
+                                const int n = (t - tb) * nkc + kc + kPrefetchW;
+                                const int tt = tb + n / nkc;
+                                if (tt < te && sub_valid(tt, r))
+                                    tma_prefetch_l2_3d(&a.map_w, 0,
+                                                       vocab0(tt, r) + static_cast<int>(prank) * (kBV / 2),
+                                                       (n % nkc) * (kKChunk / 64));
+                            }
                             int slot;
                             if (!acquire(slot)) { ok = false; break; }
                             uint8_t* st = ring + slot * kStageBytes;
                             if (a_side) {
-                                if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2u * kSStageBytes);
+                                if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2u * kStageBytes);
                                 tma_load_3d_pair(st, &a.map_h, full_leader(slot), 0, row0, kc * (kKChunk / 64));
                             } else {
                                 if (kc < a.keep_w_stages)
@@ -388,7 +369,7 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
     } else if (warp == 1) {
         // ===================================================== pair UMMA issuer (leader CTA)
         if (lane == 0 && leader) {
-            const uint32_t idesc_s = idesc_bf16_f32(2 * kTileM, kBS, false, false);
+            const uint32_t idesc_s = idesc_bf16_f32(2 * kTileM, kBV, false, false);
             const uint32_t idesc_o = idesc_bf16_f32(2 * kTileM, a.slice, true, true);
             uint32_t it = 0;
             bool ok = true;
@@ -406,7 +387,7 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 bool first = seg_first;
                 for (int q = 0; q < G; ++q) {
                     if (!sub_valid(t, q)) continue;
-                    for (int vc = 0; vc < kBS / kVChunk; ++vc) {
+                    for (int vc = 0; vc < kBV / kVChunk; ++vc) {
                         int slot;
                         if (!consume(slot)) return false;
                         const uint32_t st = smem_u32(ring + slot * kStageBytes);
@@ -430,9 +411,7 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 int ct, tb, te;
                 if (!sch.seg(j, ct, tb, te)) continue;
                 for (int t = tb; t < te && ok; ++t, ++k) {
-                    // logits buffer k & 1 was last read by the softmax for block k - 2
-                    const int sb = k & 1;
-                    if (k >= 2 && !mbar_wait(&s_free[sb], ((k >> 1) - 1) & 1, &abort_flag, a.err, kErrMmaSFree)) {
+                    if (k > 0 && !mbar_wait(&s_free, (k - 1) & 1, &abort_flag, a.err, kErrMmaSFree)) {
                         ok = false;
                         break;
                     }
@@ -446,18 +425,17 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                             for (int kk = 0; kk < kKChunk / 16; ++kk) {
                                 // K step kk: atom column kk / 4, 32-byte offset (kk % 4) inside the swizzled row
                                 const uint32_t ko = (kk >> 2) * kAtomCol + (kk & 3) * 32;
-                                const uint32_t kw = (kk >> 2) * kAtomColW + (kk & 3) * 32;
                                 const uint64_t ad = smem_desc(st + ko, 16, 1024, kSwizzle128B);
-                                const uint64_t bd = smem_desc(st + kHalfB + kw, 16, 1024, kSwizzle128B);
-                                umma_ss_pair(tmem + kTmemS + sb * kBS, ad, bd, idesc_s, (kc | kk) != 0 ? 1u : 0u);
+                                const uint64_t bd = smem_desc(st + kHalfB + ko, 16, 1024, kSwizzle128B);
+                                umma_ss_pair(tmem + kTmemS, ad, bd, idesc_s, (kc | kk) != 0 ? 1u : 0u);
                             }
                             umma_commit_pair(&empty_bar[slot], 0x3);
                         }
                         if (!ok) break;
-                        umma_commit_pair(&s_full[sb], 0x3);
+                        umma_commit_pair(&s_full, 0x3);
                     } else {
-                        mbar_arrive_remote(&s_full[sb], 0);
-                        mbar_arrive_remote(&s_full[sb], 1);
+                        mbar_arrive_remote(&s_full, 0);
+                        mbar_arrive_remote(&s_full, 1);
                     }
                     if (t > tb) ok = do_o(k - 1, t - 1, t - 1 == tb);
                 }
@@ -503,9 +481,7 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
             }
             for (int t = tb; t < te; ++t, ++k) {
                 const bool valid = sub_valid(t, r);
-                const int sb = k & 1;
-                const uint32_t s_col = kTmemS + static_cast<uint32_t>(sb) * kBS;
-                mbar_wait(&s_full[sb], (k >> 1) & 1, &abort_flag, a.err, kErrSmaxSFull);
+                mbar_wait(&s_full, k & 1, &abort_flag, a.err, kErrSmaxSFull);
                 softmax_bar();
                 if (abort_flag) { ok = false; break; }
                 tc_fence_after();
@@ -513,9 +489,9 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 float smax = -INFINITY;
                 if (valid) {
 #pragma unroll 1
-                    for (int c0 = 0; c0 < kBS; c0 += 64) {
+                    for (int c0 = 0; c0 < kBV; c0 += 64) {
                         uint32_t v[64];
-                        tmem_ld64(tmem + s_col + lane_addr + c0, v);
+                        tmem_ld64(tmem + kTmemS + lane_addr + c0, v);
 #pragma unroll
                         for (int i = 0; i < 64; ++i) smax = fmaxf(smax, __uint_as_float(v[i]));
                     }
@@ -551,14 +527,14 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 // are contiguous: lanes 2m and 2m+1 swap one value per column pair and
                 // each stores the two rows (2m, 2m+1) of one column as a bf16 pair.
                 if (valid) {
-                    __nv_bfloat16* pt = a.pbuf + static_cast<size_t>((g * 2 + (k & 1)) * G + r) * kBS * kCanvas;
+                    __nv_bfloat16* pt = a.pbuf + static_cast<size_t>((g * 2 + (k & 1)) * G + r) * kBV * kCanvas;
                     const bool odd = lane & 1;
                     const int prow = crow & ~1;
                     const int v0 = vocab0(t, r) + a.vocab_offset;     // global vocabulary index of column 0
 #pragma unroll 1
-                    for (int c0 = 0; c0 < kBS; c0 += 64) {
+                    for (int c0 = 0; c0 < kBV; c0 += 64) {
                         uint32_t v[64];
-                        tmem_ld64(tmem + s_col + lane_addr + c0, v);
+                        tmem_ld64(tmem + kTmemS + lane_addr + c0, v);
                         float lc = 0.f;            // this 64-entry chunk's mass, relative to m_ref
 #pragma unroll
                         for (int i = 0; i < 64; i += 2) {
@@ -609,7 +585,7 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 softmax_bar();
                 const bool resc = rescale_any != 0;
                 if (sleader) {
-                    mbar_arrive_remote(&s_free[sb], 0);
+                    mbar_arrive_remote(&s_free, 0);
                     red_release_add(cnt_p, 1u);
                 }
                 // --- O of block k-1 must be complete before block k may accumulate (and be rescaled)
@@ -757,7 +733,7 @@ __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
     const int tid = threadIdx.x;
     const bool head = blockIdx.y == 0;      // writes the per-position scalars
     if (blockIdx.x == 0 && head) {
-        for (int i = tid; i < counter_words(a.n_groups); i += blockDim.x) a.counters[i] = 0u;
+        for (int i = tid; i < a.n_groups * 128; i += blockDim.x) a.counters[i] = 0u;
     }
     if (tid == 0) {
         sh_skip = a.stop[c] != 0;

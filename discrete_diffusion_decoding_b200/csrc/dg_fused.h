@@ -30,8 +30,6 @@ struct FusedArgs {
     int32_t* sidx;
     int step;
     int C, V, d, G, slice, n_groups, steps_per_tile, max_seg;
-    int n_pairs;         // CTA pairs in the grid (every resident pair; pairs beyond n_groups * G idle)
-    int placement;       // 0: roles by cluster index; 1: every group within one half of the SM ids
     int vocab_offset;    // vocabulary index of row 0 of W / E (a shard of the vocabulary; 0 otherwise):
                          // added to the argmax and sample indices and to the sampled mode's chunk counter
     int keep_w_stages;   // E aliases W: the first keep_w_stages hidden-column stages of every W

@@ -92,7 +92,7 @@ extern "C" dg_status dg_denoise_stats_noalloc(const dg_params* p, int step, cons
     uint8_t* base = static_cast<uint8_t*>(ws);
     dg_noalloc_clear_kernel<<<4, 256, 0, s>>>(reinterpret_cast<int32_t*>(base + L.stop), pl.C,
                                               reinterpret_cast<int32_t*>(base + L.err),
-                                              reinterpret_cast<uint32_t*>(base + L.counters), counter_words(pl.n_groups));
+                                              reinterpret_cast<uint32_t*>(base + L.counters), pl.n_groups * 128);
     if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
 
     // statistics only: no seeds, no sampler state, and the argmax mode (no sample is drawn)
