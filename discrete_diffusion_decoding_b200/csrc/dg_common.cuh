@@ -27,19 +27,6 @@ constexpr int kFusedStageBytes = 64 * 1024;
 #define DG_KEEP_W_TENTHS 3
 #endif
 constexpr int kKeepWTenths = DG_KEEP_W_TENTHS;
-// L2 prefetch distances of the fused kernel's streamed operands, in pipeline loads: the W
-// box this many loads ahead in the logits stream, and the E box this many loads ahead in
-// the self-conditioning stream, are requested into L2 when a load is issued, so that the
-// loads themselves find their bytes on chip (the three shared-memory stages alone cannot
-// cover DRAM latency at the full SM clock).
-#ifndef DG_PREFETCH_W
-#define DG_PREFETCH_W 8
-#endif
-#ifndef DG_PREFETCH_E
-#define DG_PREFETCH_E 8
-#endif
-constexpr int kPrefetchW = DG_PREFETCH_W;
-constexpr int kPrefetchE = DG_PREFETCH_E;
 constexpr int kFusedSmemBytes = kFusedStages * kFusedStageBytes + 1024 + 4 * kMaxCanvas;
 constexpr float kLazyRescale = 8.0f;  // log2 units the shared reference may lag the running max
 

@@ -270,20 +270,6 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 return true;
             };
             const int nkc = a.d / kKChunk;                 // logits stages per W tile
-            const int ne = 2 * G;                          // self-conditioning E loads per block (full blocks)
-            // B side: the E box of load n of block t's self-conditioning stream (n may run into block t + 1)
-            auto prefetch_e = [&](int t, int n, int te) {
-                if (kPrefetchE <= 0) return;
-                while (n >= ne) {
-                    n -= ne;
-                    ++t;
-                }
-                const int q = n >> 1, vc = n & 1;
-                if (t < te && sub_valid(t, q))
-                    tma_prefetch_l2_3d(&a.map_e, 0, vocab0(t, q) + vc * kVChunk,
-                                       (d0 + static_cast<int>(prank) * (a.slice / 2)) / 64);
-            };
-            int piece_te = 0;
             auto emit_o = [&](int k, int t) -> bool {
                 if (a_side) {
                     if (!wait_counter(cnt_p, static_cast<uint32_t>(nG2 * (k + 1)), &abort_flag, a.err, kErrProducerP))
@@ -304,7 +290,6 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                             tma_load_3d_pair(st, &a.map_p, full_leader(slot), 0, prow + vc * kVChunk,
                                              static_cast<int>(prank) * 2);
                         } else {
-                            prefetch_e(t, q * 2 + vc + kPrefetchE, piece_te);
                             // this CTA's half of the column slice (n_ech atoms of 64 columns) in one 3-D box
                             tma_load_3d_pair_hint(st + kHalfB, &a.map_e, full_leader(slot), 0,
                                                   vocab0(t, q) + vc * kVChunk,
@@ -319,20 +304,10 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 int ct, tb, te;
                 if (!sch.seg(j, ct, tb, te)) continue;
                 const int row0 = active[ct] * kCanvas + static_cast<int>(prank) * kTileM;
-                piece_te = te;
                 for (int t = tb; t < te && ok; ++t, ++k) {
                     if (sub_valid(t, r)) {
                         const int v0 = vocab0(t, r) + static_cast<int>(prank) * (kBV / 2);
                         for (int kc = 0; kc < nkc; ++kc) {
-                            if (!a_side && kPrefetchW > 0) {
-                                // the W box kPrefetchW loads ahead in this piece's logits stream
-                                const int n = (t - tb) * nkc + kc + kPrefetchW;
-                                const int tt = tb + n / nkc;
-                                if (tt < te && sub_valid(tt, r))
-                                    tma_prefetch_l2_3d(&a.map_w, 0,
-                                                       vocab0(tt, r) + static_cast<int>(prank) * (kBV / 2),
-                                                       (n % nkc) * (kKChunk / 64));
-                            }
                             int slot;
                             if (!acquire(slot)) { ok = false; break; }
                             uint8_t* st = ring + slot * kStageBytes;

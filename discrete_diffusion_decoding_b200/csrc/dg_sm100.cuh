@@ -274,15 +274,6 @@ __device__ __forceinline__ void tma_load_3d_pair_hint(void* dst, const CUtensorM
         : "memory");
 }
 
-// Prefetch the box at {x, y, z} of a 3-D tensor map into L2 (no shared memory, no barrier):
-// brings a later load's bytes on chip early so that the load itself hits L2.
-__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int x, int y, int z) {
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(x), "r"(y), "r"(z)
-                 : "memory");
-}
-
 // Cache policy for data read once: its L2 lines are the first candidates for eviction.
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t pol;
