@@ -16,7 +16,8 @@ from ._abi import DgError, DgParams, check, lib
 __all__ = ["DgError", "DgParams", "params", "workspace_size", "plan", "temperature", "dg_canvas_init",
            "dg_denoise_step", "dg_stop_check", "dg_stub_hidden", "last_launch_count", "profile_enable",
            "profile_collect", "dg_denoise_stats_noalloc", "dg_debug_set_error", "Workspace", "StepBuffers",
-           "decode_batch", "decode_block_ar", "dg_partial_bytes", "dg_denoise_partial", "dg_denoise_merge"]
+           "decode_batch", "decode_block_ar", "dg_partial_bytes", "dg_denoise_partial", "dg_denoise_merge",
+           "dg_debug_set_counter_wait_limit"]
 
 
 def params(n_canvas, vocab, hidden, **overrides):
@@ -113,6 +114,11 @@ def dg_debug_set_error(p, ws, code, stream=None):
     """Host-side fault injection: write `code` into the workspace's device error word."""
     check("dg_debug_set_error", lib().dg_debug_set_error(ctypes.byref(p), ws.ptr, ws.nbytes, int(code),
                                                          _stream(stream)))
+
+
+def dg_debug_set_counter_wait_limit(ns):
+    """Testing hook: limit the fused kernel's waits on other CTAs' counters to ns (0: the 2 s default)."""
+    check("dg_debug_set_counter_wait_limit", lib().dg_debug_set_counter_wait_limit(int(ns)))
 
 
 def dg_denoise_stats_noalloc(p, step, h, W, E, entropy, argmax, lse, selfcond, stream=None):

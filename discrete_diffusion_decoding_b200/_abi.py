@@ -12,7 +12,7 @@ DG_OK, DG_EINVAL, DG_ECUDA, DG_EUNSUPPORTED, DG_ETIMEOUT, DG_ENOMEM = 0, -1, -2,
 EXPORTS = ("dg_params_default", "dg_temperature", "dg_workspace_size", "dg_canvas_init", "dg_denoise_step",
            "dg_stop_check", "dg_stub_hidden", "dg_status_string", "dg_last_launch_count", "dg_plan",
            "dg_profile_enable", "dg_profile_collect", "dg_denoise_stats_noalloc", "dg_debug_set_error",
-           "dg_partial_bytes", "dg_denoise_partial", "dg_denoise_merge")
+           "dg_partial_bytes", "dg_denoise_partial", "dg_denoise_merge", "dg_debug_set_counter_wait_limit")
 
 
 class DgParams(ctypes.Structure):
@@ -72,6 +72,8 @@ def lib():
         L.dg_denoise_partial.restype = i32
         L.dg_denoise_merge.argtypes = [P, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.dg_denoise_merge.restype = i32
+        L.dg_debug_set_counter_wait_limit.argtypes = [ctypes.c_ulonglong]
+        L.dg_debug_set_counter_wait_limit.restype = i32
         L.dg_profile_enable.argtypes = [i32]
         L.dg_profile_enable.restype = i32
         L.dg_profile_collect.argtypes = [ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_float),

@@ -12,6 +12,7 @@
 #include "dg_common.cuh"
 #include "dg_fused.h"
 #include "dg_host.h"
+#include "dg_sm100.cuh"
 
 using namespace dg;
 
@@ -23,6 +24,7 @@ namespace {
 constexpr int kFusedSmem = kFusedSmemBytes;
 constexpr int kMaxDevices = 64;
 thread_local int g_last_launches = 0;
+thread_local unsigned long long g_counter_wait_ns = DG_WAIT_LIMIT_NS;
 
 // Event pairs recorded around fused-kernel launches while profiling is enabled.
 struct ProfileState {
@@ -250,6 +252,7 @@ dg_status launch_fused_and_combine(const dg_params* p, const Plan& pl, const Lay
     fa.steps_per_tile = (io.vocab_rows + pl.group * kBV - 1) / (pl.group * kBV);
     fa.max_seg = pl.max_seg;
     fa.scale_log2 = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
+    fa.counter_wait_ns = g_counter_wait_ns;
 
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
@@ -541,6 +544,11 @@ dg_status dg_denoise_merge(const dg_params* p, int step, int n_parts, const void
     st = launch_stop(p, pl, L, workspace_dev, step, seeds_dev, tokens_dev, entropy_dev, argmax_dev, accept_dev, s);
     if (st != DG_OK) return st;
     g_last_launches = 2;
+    return DG_OK;
+}
+
+dg_status dg_debug_set_counter_wait_limit(unsigned long long ns) {
+    g_counter_wait_ns = ns == 0 ? DG_WAIT_LIMIT_NS : ns;
     return DG_OK;
 }
 

@@ -19,15 +19,26 @@ constexpr int kMaxSlice = 256;    // widest self-conditioning column slice a CTA
 constexpr int kMaxCanvas = 256;   // canvases per call (the fused kernel keeps the active list in shared memory)
 constexpr int kMaxParts = 64;     // vocabulary shards one dg_denoise_merge call takes
 constexpr int kThreads = 256;     // threads of the fused kernel
-constexpr int kFusedStages = 3;   // TMA ring stages of the fused kernel
-constexpr int kFusedStageBytes = 64 * 1024;
+// The fused kernel's operand rings: every pipeline stage is one A box (h rows or P^T
+// columns, both read from L2) and one B box (W rows or E columns, mostly from DRAM), each
+// 32 KB per CTA; the B ring is one stage deeper so that more of the DRAM-bound operand is
+// in flight.
+#ifndef DG_A_STAGES
+#define DG_A_STAGES 3
+#endif
+#ifndef DG_B_STAGES
+#define DG_B_STAGES 4
+#endif
+constexpr int kAStages = DG_A_STAGES;
+constexpr int kBStages = DG_B_STAGES;
+constexpr int kRingBoxBytes = 32 * 1024;
 // With E aliasing W, this many tenths of the hidden columns of every W tile keep normal
 // L2 priority between the logits and the self-conditioning pass (the rest is streamed).
 #ifndef DG_KEEP_W_TENTHS
 #define DG_KEEP_W_TENTHS 3
 #endif
 constexpr int kKeepWTenths = DG_KEEP_W_TENTHS;
-constexpr int kFusedSmemBytes = kFusedStages * kFusedStageBytes + 1024 + 4 * kMaxCanvas;
+constexpr int kFusedSmemBytes = (kAStages + kBStages) * kRingBoxBytes + 1024 + 4 * kMaxCanvas;
 constexpr float kLazyRescale = 8.0f;  // log2 units the shared reference may lag the running max
 
 // ------------------------------------------------------------------ Philox4x32-10

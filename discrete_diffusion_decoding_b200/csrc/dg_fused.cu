@@ -54,9 +54,7 @@ namespace dg {
 
 namespace {
 
-constexpr int kStages = kFusedStages;
-constexpr int kStageBytes = kFusedStageBytes;   // per CTA: A operand 32 KB + B operand half 32 KB
-constexpr int kHalfB = 32 * 1024;
+constexpr int kBox = kRingBoxBytes;              // one A or B box per CTA per stage
 constexpr uint32_t kAtomCol = 128u * 128u;     // bytes of one 64-column swizzle atom column of a 128-row box
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 0;             // logits tile columns [0, 256)
@@ -81,8 +79,11 @@ __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Bounded poll until *ctr >= target (wrap-safe comparison).
-__device__ bool wait_counter(const uint32_t* ctr, uint32_t target, volatile int* abort, int* err, int code) {
+// Bounded poll until *ctr >= target (wrap-safe comparison): the waits on other CTAs of
+// the group, limited by limit_ns (a kernel argument; the waits that drain this CTA's
+// own loads and UMMAs keep the fixed DG_WAIT_LIMIT_NS).
+__device__ bool wait_counter(const uint32_t* ctr, uint32_t target, volatile int* abort, int* err, int code,
+                             uint64_t limit_ns) {
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
         if (static_cast<int32_t>(ld_acquire_u32(ctr) - target) >= 0) return true;
@@ -91,9 +92,9 @@ __device__ bool wait_counter(const uint32_t* ctr, uint32_t target, volatile int*
             const uint64_t now = global_ns();
             if (it == 0) {
                 t0 = now;
-            } else if (now - t0 > DG_WAIT_LIMIT_NS) {
+            } else if (now - t0 > limit_ns) {
                 atomicCAS(err, 0, code);
-                *abort = 1;
+                raise_pair_abort(abort);
                 return false;
             }
         }
@@ -174,10 +175,12 @@ __device__ __forceinline__ float neg_log2_uniform(uint32_t w) {
 template <bool kSample>
 __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    int* active = reinterpret_cast<int*>(ring + kStages * kStageBytes);
+    uint8_t* a_ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* b_ring = a_ring + kAStages * kBox;
+    int* active = reinterpret_cast<int*>(b_ring + kBStages * kBox);
 
-    __shared__ uint64_t full_bar[kStages], empty_bar[kStages];
+    // a_* / b_*: the A and B rings' barriers (full: the leader's, counting both CTAs' bytes)
+    __shared__ uint64_t a_full[kAStages], a_empty[kAStages], b_full[kBStages], b_empty[kBStages];
     __shared__ uint64_t s_full, s_free, o_ready, o_done, drain_bar;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
@@ -196,9 +199,13 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
     const int d0 = r * a.slice;
 
     if (tid == 0) {
-        for (int i = 0; i < kStages; ++i) {
-            mbar_init(&full_bar[i], 1);      // leader: one expect_tx arrival per use, bytes of both CTAs
-            mbar_init(&empty_bar[i], 1);     // one multicast commit per use
+        for (int i = 0; i < kAStages; ++i) {
+            mbar_init(&a_full[i], 1);        // leader: one expect_tx arrival per use, bytes of both CTAs
+            mbar_init(&a_empty[i], 1);       // one multicast commit per use
+        }
+        for (int i = 0; i < kBStages; ++i) {
+            mbar_init(&b_full[i], 1);
+            mbar_init(&b_empty[i], 1);
         }
         mbar_init(&s_full, 1);
         mbar_init(&s_free, 2);               // leader: softmax of both CTAs
@@ -238,8 +245,8 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
     uint32_t* cnt_rowmax = a.counters + counter_word(g, kCntRowmax);
     uint32_t* cnt_p = a.counters + counter_word(g, kCntP);
     uint32_t* cnt_used = a.counters + counter_word(g, kCntUsed);
-    const int n_ech = a.slice / 128;                 // E boxes (64 columns each) per CTA per O stage
-    const uint32_t o_stage_bytes = 2u * kAtomCol + static_cast<uint32_t>(n_ech) * kAtomCol;   // P^T 2 x 16 KB + E
+    const int n_ech = a.slice / 128;                 // E atoms (64 columns each) per CTA per O stage
+    const uint32_t e_box_bytes = static_cast<uint32_t>(n_ech) * kAtomCol;   // <= kBox (slice <= 256)
     const int nG2 = 2 * G;                           // CTAs per group
 
     if (warp == 0 || warp == 3) {
@@ -257,14 +264,18 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
             // stages of every W tile keep normal priority (the two blocks in flight of every
             // group would not fit in L2 whole) and are read again from L2 as E
             const uint64_t pol_stream = l2_policy_evict_first();
-            // the leader's full barrier of a stage, as a shared::cluster address
-            auto full_leader = [&](int slot) { return smem_addr_in_rank(&full_bar[slot], 0); };
+            // this side's ring: its stage count, buffers and barriers
+            const int n_st = a_side ? kAStages : kBStages;
+            uint8_t* my_ring = a_side ? a_ring : b_ring;
+            uint64_t* my_full = a_side ? a_full : b_full;
+            uint64_t* my_empty = a_side ? a_empty : b_empty;
+            auto full_leader = [&](int slot) { return smem_addr_in_rank(&my_full[slot], 0); };
             uint32_t it = 0;
             bool ok = true;
             auto acquire = [&](int& slot) -> bool {
-                slot = static_cast<int>(it % kStages);
-                if (it >= kStages &&
-                    !mbar_wait(&empty_bar[slot], ((it / kStages) - 1) & 1, &abort_flag, a.err, kErrProducerEmpty))
+                slot = static_cast<int>(it % n_st);
+                if (it >= static_cast<uint32_t>(n_st) &&
+                    !mbar_wait(&my_empty[slot], ((it / n_st) - 1) & 1, &abort_flag, a.err, kErrProducerEmpty))
                     return false;
                 ++it;
                 return true;
@@ -272,7 +283,8 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
             const int nkc = a.d / kKChunk;                 // logits stages per W tile
             auto emit_o = [&](int k, int t) -> bool {
                 if (a_side) {
-                    if (!wait_counter(cnt_p, static_cast<uint32_t>(nG2 * (k + 1)), &abort_flag, a.err, kErrProducerP))
+                    if (!wait_counter(cnt_p, static_cast<uint32_t>(nG2 * (k + 1)), &abort_flag, a.err, kErrProducerP,
+                                      a.counter_wait_ns))
                         return false;
                     fence_async_global();
                 }
@@ -283,15 +295,16 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                     for (int vc = 0; vc < kBV / kVChunk; ++vc) {
                         int slot;
                         if (!acquire(slot)) return false;
-                        uint8_t* st = ring + slot * kStageBytes;
+                        uint8_t* st = my_ring + slot * kBox;
                         if (a_side) {
-                            if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2u * o_stage_bytes);
+                            if (leader) mbar_arrive_expect_tx(&my_full[slot], 2u * 2u * kAtomCol);
                             // both 64-row atoms of this CTA's canvas rows in one 3-D box
                             tma_load_3d_pair(st, &a.map_p, full_leader(slot), 0, prow + vc * kVChunk,
                                              static_cast<int>(prank) * 2);
                         } else {
+                            if (leader) mbar_arrive_expect_tx(&my_full[slot], 2u * e_box_bytes);
                             // this CTA's half of the column slice (n_ech atoms of 64 columns) in one 3-D box
-                            tma_load_3d_pair_hint(st + kHalfB, &a.map_e, full_leader(slot), 0,
+                            tma_load_3d_pair_hint(st, &a.map_e, full_leader(slot), 0,
                                                   vocab0(t, q) + vc * kVChunk,
                                                   (d0 + static_cast<int>(prank) * (a.slice / 2)) / 64, pol_stream);
                         }
@@ -310,16 +323,15 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                         for (int kc = 0; kc < nkc; ++kc) {
                             int slot;
                             if (!acquire(slot)) { ok = false; break; }
-                            uint8_t* st = ring + slot * kStageBytes;
+                            uint8_t* st = my_ring + slot * kBox;
+                            if (leader) mbar_arrive_expect_tx(&my_full[slot], 2u * kBox);
                             if (a_side) {
-                                if (leader) mbar_arrive_expect_tx(&full_bar[slot], 2u * kStageBytes);
                                 tma_load_3d_pair(st, &a.map_h, full_leader(slot), 0, row0, kc * (kKChunk / 64));
                             } else {
                                 if (kc < a.keep_w_stages)
-                                    tma_load_3d_pair(st + kHalfB, &a.map_w, full_leader(slot), 0, v0,
-                                                     kc * (kKChunk / 64));
+                                    tma_load_3d_pair(st, &a.map_w, full_leader(slot), 0, v0, kc * (kKChunk / 64));
                                 else
-                                    tma_load_3d_pair_hint(st + kHalfB, &a.map_w, full_leader(slot), 0, v0,
+                                    tma_load_3d_pair_hint(st, &a.map_w, full_leader(slot), 0, v0,
                                                           kc * (kKChunk / 64), pol_stream);
                             }
                         }
@@ -330,10 +342,10 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
             }
             // drain: every issued use of a stage has been released by the leader's
             // commit, so no load into this CTA is still in flight when it exits
-            for (uint32_t u = (it > kStages ? it - kStages : 0); u < it; ++u) {
-                const int slot = static_cast<int>(u % kStages);
+            for (uint32_t u = (it > static_cast<uint32_t>(n_st) ? it - n_st : 0); u < it; ++u) {
+                const int slot = static_cast<int>(u % n_st);
                 const uint64_t t0 = global_ns();
-                while (!mbar_try_wait(smem_u32(&empty_bar[slot]), (u / kStages) & 1)) {
+                while (!mbar_try_wait(smem_u32(&my_empty[slot]), (u / n_st) & 1)) {
                     if (global_ns() - t0 > DG_WAIT_LIMIT_NS) {
                         atomicCAS(a.err, 0, kErrProducerDrain);
                         break;
@@ -348,12 +360,22 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
             const uint32_t idesc_o = idesc_bf16_f32(2 * kTileM, a.slice, true, true);
             uint32_t it = 0;
             bool ok = true;
-            auto consume = [&](int& slot) -> bool {
-                slot = static_cast<int>(it % kStages);
-                if (!mbar_wait(&full_bar[slot], (it / kStages) & 1, &abort_flag, a.err, kErrMmaFull)) return false;
+            // stage `it`: A box in A-ring slot it % kAStages, B box in B-ring slot it % kBStages
+            int sa = 0, sb = 0;
+            auto consume = [&](uint32_t& a_addr, uint32_t& b_addr) -> bool {
+                sa = static_cast<int>(it % kAStages);
+                sb = static_cast<int>(it % kBStages);
+                if (!mbar_wait(&a_full[sa], (it / kAStages) & 1, &abort_flag, a.err, kErrMmaFull)) return false;
+                if (!mbar_wait(&b_full[sb], (it / kBStages) & 1, &abort_flag, a.err, kErrMmaFull)) return false;
                 ++it;
                 tc_fence_after();
+                a_addr = smem_u32(a_ring + sa * kBox);
+                b_addr = smem_u32(b_ring + sb * kBox);
                 return true;
+            };
+            auto release = [&]() {
+                umma_commit_pair(&a_empty[sa], 0x3);
+                umma_commit_pair(&b_empty[sb], 0x3);
             };
             // seg_first: block t is the first of its piece, so O starts from zero
             auto do_o = [&](int k, int t, bool seg_first) -> bool {
@@ -363,17 +385,16 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 for (int q = 0; q < G; ++q) {
                     if (!sub_valid(t, q)) continue;
                     for (int vc = 0; vc < kBV / kVChunk; ++vc) {
-                        int slot;
-                        if (!consume(slot)) return false;
-                        const uint32_t st = smem_u32(ring + slot * kStageBytes);
+                        uint32_t sta, stb;
+                        if (!consume(sta, stb)) return false;
 #pragma unroll
                         for (int kk = 0; kk < kVChunk / 16; ++kk) {
-                            const uint64_t ad = smem_desc(st + kk * 2048, kAtomCol, 1024, kSwizzle128B);
-                            const uint64_t bd = smem_desc(st + kHalfB + kk * 2048, kAtomCol, 1024, kSwizzle128B);
+                            const uint64_t ad = smem_desc(sta + kk * 2048, kAtomCol, 1024, kSwizzle128B);
+                            const uint64_t bd = smem_desc(stb + kk * 2048, kAtomCol, 1024, kSwizzle128B);
                             umma_ss_pair(tmem + kTmemO, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
                         }
                         first = false;
-                        umma_commit_pair(&empty_bar[slot], 0x3);
+                        release();
                     }
                 }
                 // every P tile of block k has landed in both CTAs' shared memory
@@ -393,18 +414,17 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                     tc_fence_after();
                     if (sub_valid(t, r)) {
                         for (int kc = 0; kc < a.d / kKChunk; ++kc) {
-                            int slot;
-                            if (!consume(slot)) { ok = false; break; }
-                            const uint32_t st = smem_u32(ring + slot * kStageBytes);
+                            uint32_t sta, stb;
+                            if (!consume(sta, stb)) { ok = false; break; }
 #pragma unroll
                             for (int kk = 0; kk < kKChunk / 16; ++kk) {
                                 // K step kk: atom column kk / 4, 32-byte offset (kk % 4) inside the swizzled row
                                 const uint32_t ko = (kk >> 2) * kAtomCol + (kk & 3) * 32;
-                                const uint64_t ad = smem_desc(st + ko, 16, 1024, kSwizzle128B);
-                                const uint64_t bd = smem_desc(st + kHalfB + ko, 16, 1024, kSwizzle128B);
+                                const uint64_t ad = smem_desc(sta + ko, 16, 1024, kSwizzle128B);
+                                const uint64_t bd = smem_desc(stb + ko, 16, 1024, kSwizzle128B);
                                 umma_ss_pair(tmem + kTmemS, ad, bd, idesc_s, (kc | kk) != 0 ? 1u : 0u);
                             }
-                            umma_commit_pair(&empty_bar[slot], 0x3);
+                            release();
                         }
                         if (!ok) break;
                         umma_commit_pair(&s_full, 0x3);
@@ -478,10 +498,11 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 if (sleader) {
                     red_release_add(cnt_rowmax, 1u);
                     const bool w = wait_counter(cnt_rowmax, static_cast<uint32_t>(nG2 * (k + 1)), &abort_flag,
-                                                a.err, kErrSmaxRowmax);
+                                                a.err, kErrSmaxRowmax, a.counter_wait_ns);
                     // P buffer (k & 1) was last read for block k-2
                     if (w && k >= 2)
-                        wait_counter(cnt_used, static_cast<uint32_t>(G * (k - 1)), &abort_flag, a.err, kErrSmaxUsed);
+                        wait_counter(cnt_used, static_cast<uint32_t>(G * (k - 1)), &abort_flag, a.err, kErrSmaxUsed,
+                                     a.counter_wait_ns);
                 }
                 softmax_bar();
                 if (abort_flag) { ok = false; break; }

@@ -36,6 +36,7 @@ struct FusedArgs {
                          // tile keep normal L2 priority, so the self-conditioning pass finds them
                          // there (0 when E is a separate matrix)
     float scale_log2;    // log2(e) / T
+    unsigned long long counter_wait_ns;   // limit of the waits on other CTAs' counters (the drains keep theirs)
 };
 
 struct CombineArgs {

@@ -118,9 +118,21 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
     return ok != 0;
 }
 
+// Raise the abort flag of this CTA and of the other CTA of its pair (same shared-memory
+// offset in cluster rank ctarank ^ 1): both CTAs then leave their loops together.  Only
+// valid in a kernel of 2-CTA clusters, between its first and last cluster barrier.
+__device__ __forceinline__ void raise_pair_abort(volatile int* abort) {
+    *abort = 1;
+    uint32_t local = smem_u32(const_cast<int*>(abort)), remote;
+    uint32_t rank;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank ^ 1u));
+    asm volatile("st.volatile.shared::cluster.u32 [%0], %1;" ::"r"(remote), "r"(1u) : "memory");
+}
+
 // Bounded wait for the phase with the given parity to complete.  On timeout, or
 // when another role has already raised `abort`, records `code` in *err (first
-// error wins), raises *abort and returns false.
+// error wins), raises the pair's abort flags and returns false.
 template <bool kClusterAcquire = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* err, int code) {
@@ -133,7 +145,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         if (*abort) return false;
         if (global_ns() - t0 > DG_WAIT_LIMIT_NS) {
             atomicCAS(err, 0, code);
-            *abort = 1;
+            raise_pair_abort(abort);
             return false;
         }
     }

@@ -182,6 +182,17 @@ dg_status dg_debug_set_error(const dg_params* p, void* workspace_dev, size_t wor
                              void* stream);
 
 /*
+ * Testing hook for the timeout path (not on the pages): the fused kernel launched by later
+ * calls on this host thread limits each of its waits on other CTAs' progress counters (the
+ * row-maximum exchange and the probability tiles of the group) to `ns` nanoseconds instead
+ * of 2 s; 0 restores 2 s.  A wait that runs out makes the kernel leave early and record
+ * the error word exactly as a stalled peer would (DG_ETIMEOUT from dg_stop_check, poisoned
+ * results).  The waits that drain a CTA's own loads and tensor-core operations keep their
+ * 2 s limit, so none is in flight when a CTA leaves.  Always returns DG_OK.
+ */
+dg_status dg_debug_set_counter_wait_limit(unsigned long long ns);
+
+/*
  * Benchmark-only stand-in for the denoiser network (not on the pages):
  *   h_i = gain * (a E[tgt_i] + (1 - a) E[x_i]) + noise * n_i,   a = s / max_steps,
  * tgt_i uniform over V (Philox tag 2, step 0), n_i standard normal by Box-Muller on
