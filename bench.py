@@ -34,6 +34,7 @@ V, D, N_POS, STEP, BOUND = 262144, 2816, 256, 1, 0.1
 ACCEPT_MODE = 0            # 0: accepted positions keep the argmax; 1: a Gumbel-max sample (--accept sample)
 ACCEPT_RULE = 0            # 0: accept every position with H <= bound; 1: by groups (--rule group)
 CANVASES, UNTIED = 1, False  # per rank; other values are context measurements (--canvases, --untied)
+LOGITS_FP8 = False         # --logits e4m3: the head as E4M3 codes for the logits GEMM (its own bench line)
 METRIC = "canvas positions/s per denoise step (V=262144,d=2816); % of roofline"
 WORKLOAD = ("single-step microbenchmark: 1 canvas of 256 positions, V=262144, d=2816, tied bf16 E=W ~N(0,0.02), "
             "hidden bf16 N(0,1)/sqrt(d)*8, step 1 (T=0.8), bound 0.1; outputs tokens/H/argmax/accept/self-cond fp32")
@@ -221,6 +222,15 @@ def _set_shape(canvases, untied):
         WORKLOAD = WORKLOAD.replace("tied bf16 E=W ~N(0,0.02)", "untied bf16 W, E ~N(0,0.02) (context measurement)")
 
 
+def _set_logits(fp8):
+    """--logits e4m3: E4M3 logits operands, bf16 self-conditioning (the low-precision head option)."""
+    global LOGITS_FP8, WORKLOAD
+    LOGITS_FP8 = bool(fp8)
+    if LOGITS_FP8:
+        WORKLOAD = WORKLOAD.replace("tied bf16 E=W ~N(0,0.02)", "head ~N(0,0.02) as E4M3 codes with one power-of-two "
+                                    "scale for the logits GEMM, its exact bf16 decoding as E")
+
+
 def _set_accept(mode, rule=0):
     """--accept sample / --rule group: time the sampled-acceptance kernel or the group rule."""
     global ACCEPT_MODE, ACCEPT_RULE, WORKLOAD
@@ -379,6 +389,11 @@ def run_gpu(args):
         W = W_host.to(dev)
         E = synth.weights(V, D, seed=1235).to(dev) if UNTIED else W
     del W_host
+    w_exp = 0
+    if LOGITS_FP8:
+        # one-time head preparation: E4M3 codes on the GPU, and their exact bf16 decoding as E
+        W, w_exp = dg.quantize_head_e4m3(W)
+        E = (W.view(torch.float8_e4m3fn).to(torch.float32) * (2.0 ** w_exp)).to(torch.bfloat16)
     h_host = synth.gaussian_hidden(N_POS, D, seed=42)
     if world > 1:
         tdist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
@@ -386,7 +401,8 @@ def run_gpu(args):
     # replicas: every rank owns CANVASES canvases of its own (seed = the global canvas index);
     # vocabulary split: every rank works on the same canvases over its rows of the head
     c0 = 0 if split else shard_canvases(world * CANVASES, rank, world)[0]
-    p = dg.params(CANVASES, V, D, accept_mode=ACCEPT_MODE, accept_rule=ACCEPT_RULE, tied=0 if UNTIED else 1)
+    p = dg.params(CANVASES, V, D, accept_mode=ACCEPT_MODE, accept_rule=ACCEPT_RULE,
+                  tied=0 if (UNTIED or LOGITS_FP8) else 1, logits_format=1 if LOGITS_FP8 else 0, w_scale_exp=w_exp)
     bufs = dg.StepBuffers(p, dev)
     seeds = torch.arange(c0, c0 + CANVASES, dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream()
@@ -509,16 +525,24 @@ def run_gpu(args):
         achieved = flops_launch / (k1_max * 1e-3) / 1e12
         hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])) * 1e9
         bytes_launch = (2.0 if UNTIED else 1.0) * 2.0 * rows_per_rank * D
+        if LOGITS_FP8:
+            # half the FLOPs at the E4M3 rate (twice bf16, the nominal ratio), half at the bf16 rate:
+            # the launch's peak is 4 / (1/2 + 1) / 2 = 4/3 of the bf16 figure; bytes: 1-byte codes + bf16 E
+            fp8_gain = 4.0 / 3.0
+            peak_tf, peak_burst, peak_sus = peak_tf * fp8_gain, peak_burst * fp8_gain, peak_sus * fp8_gain
+            bytes_launch = 3.0 * rows_per_rank * D
         roof_ms = max(flops_launch / (peak_tf * 1e12), bytes_launch / hbm) * 1e3
         # the committed DRAM capture is of the default kernel on the one-canvas tied workload
-        traffic = profiled_traffic() if (ACCEPT_MODE == 0 and CANVASES == 1 and not UNTIED and not split) else None
+        traffic = profiled_traffic() if (ACCEPT_MODE == 0 and CANVASES == 1 and not UNTIED and not split
+                                         and not LOGITS_FP8) else None
         positions = (1 if split else world) * N_POS
         value = positions / (ms_per_step * 1e-3)
         line = {
             "metric": METRIC, "value": value, "unit": "positions/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "strong" if split else "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "e4m3 logits + bf16 self-conditioning" if LOGITS_FP8 else "bf16",
+            "data": "synthetic",
             "config": {"workload": WORKLOAD, "n_canvas": (1 if split else world) * CANVASES, "positions": positions,
                        "vocab": V, "hidden": D,
                        "parallelism": (f"vocabulary split x{world} (all-gather of shard partials)" if split else
@@ -528,7 +552,8 @@ def run_gpu(args):
             "steps_per_s": 1e3 / ms_per_step,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": achieved / peak_tf, "traffic": traffic,
-                         "kernel": "dg_fused_sample_kernel" if ACCEPT_MODE else "dg_fused_kernel",
+                         "kernel": ("dg_fused_fp8" if LOGITS_FP8 else "dg_fused") + ("_sample_kernel" if ACCEPT_MODE
+                                                                                       else "_kernel"),
                          "kernel_ms": k1_max, "launches_timed": n_k1, "flops_per_launch": flops_launch,
                          "peak_regime": regime,
                          "peak_source": (f"{peaks_src} bf16 {regime}: " +
@@ -546,7 +571,10 @@ def run_gpu(args):
         }
         if split:
             line["multi_gpu_note"] = "vocabulary split: NCCL all-gather of each rank's partial, merge on every rank"
-        if world == 1 and not args.no_cpu_baseline and CANVASES == 1 and not UNTIED:
+        if LOGITS_FP8:
+            line["roofline"]["peak_source"] += (" x 4/3: the logits GEMM runs on E4M3 operands at twice the bf16 "
+                                                "rate (nominal ratio), the self-conditioning GEMM at the bf16 rate")
+        if world == 1 and not args.no_cpu_baseline and CANVASES == 1 and not UNTIED and not LOGITS_FP8:
             # bounded sample of the same workload through the float64 oracle on the host cores
             from oracle import stage
             W64 = stage.bf16_to_f64(synth.bf16_bits(W.cpu()))
@@ -580,6 +608,8 @@ def main(argv=None):
     ap.add_argument("--canvases", type=int, default=1,
                     help="canvases per rank in one launch; values other than 1 are context measurements, not bench lines")
     ap.add_argument("--untied", action="store_true", help="separate W and E (context measurement, not a bench line)")
+    ap.add_argument("--logits", choices=["bf16", "e4m3"], default="bf16",
+                    help="number format of the logits GEMM operands (e4m3: the head as 8-bit codes; its own bench line)")
     ap.add_argument("--split", choices=["replicas", "vocab"], default="replicas",
                     help="with --gpus N > 1: independent replicas (weak scaling, default) or one head split by "
                          "vocabulary rows over the ranks (strong scaling)")
@@ -590,6 +620,7 @@ def main(argv=None):
         _set_vocab(args.vocab)
     _set_accept(1 if args.accept == "sample" else 0, 1 if args.rule == "group" else 0)
     _set_shape(args.canvases, args.untied)
+    _set_logits(args.logits == "e4m3")
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.cpu_configs:

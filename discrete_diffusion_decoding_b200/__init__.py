@@ -17,7 +17,7 @@ __all__ = ["DgError", "DgParams", "params", "workspace_size", "plan", "temperatu
            "dg_denoise_step", "dg_stop_check", "dg_stub_hidden", "last_launch_count", "profile_enable",
            "profile_collect", "dg_denoise_stats_noalloc", "dg_debug_set_error", "Workspace", "StepBuffers",
            "decode_batch", "decode_block_ar", "dg_partial_bytes", "dg_denoise_partial", "dg_denoise_merge",
-           "dg_debug_set_counter_wait_limit"]
+           "dg_debug_set_counter_wait_limit", "dg_quantize_e4m3", "quantize_head_e4m3"]
 
 
 def params(n_canvas, vocab, hidden, **overrides):
@@ -114,6 +114,24 @@ def dg_debug_set_error(p, ws, code, stream=None):
     """Host-side fault injection: write `code` into the workspace's device error word."""
     check("dg_debug_set_error", lib().dg_debug_set_error(ctypes.byref(p), ws.ptr, ws.nbytes, int(code),
                                                          _stream(stream)))
+
+
+def dg_quantize_e4m3(src, codes, exps, per_row, stream=None):
+    """E4M3 codes of a bf16 matrix with power-of-two scales (per row, or one for the tensor)."""
+    rows, cols = src.shape
+    check("dg_quantize_e4m3", lib().dg_quantize_e4m3(_ptr(src), int(rows), int(cols), int(per_row), _ptr(codes),
+                                                     _ptr(exps), _stream(stream)))
+
+
+def quantize_head_e4m3(W, stream=None):
+    """The head as E4M3 codes with one power-of-two scale: returns (codes uint8 [V, d], exponent int).
+
+    Synchronises the stream to read the exponent (a one-time step when a head is loaded).
+    """
+    codes = torch.empty(W.shape, dtype=torch.uint8, device=W.device)
+    exps = torch.empty(1, dtype=torch.int32, device=W.device)
+    dg_quantize_e4m3(W, codes, exps, 0, stream)
+    return codes, int(exps.item())
 
 
 def dg_debug_set_counter_wait_limit(ns):

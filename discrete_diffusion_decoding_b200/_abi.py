@@ -12,7 +12,8 @@ DG_OK, DG_EINVAL, DG_ECUDA, DG_EUNSUPPORTED, DG_ETIMEOUT, DG_ENOMEM = 0, -1, -2,
 EXPORTS = ("dg_params_default", "dg_temperature", "dg_workspace_size", "dg_canvas_init", "dg_denoise_step",
            "dg_stop_check", "dg_stub_hidden", "dg_status_string", "dg_last_launch_count", "dg_plan",
            "dg_profile_enable", "dg_profile_collect", "dg_denoise_stats_noalloc", "dg_debug_set_error",
-           "dg_partial_bytes", "dg_denoise_partial", "dg_denoise_merge", "dg_debug_set_counter_wait_limit")
+           "dg_partial_bytes", "dg_denoise_partial", "dg_denoise_merge", "dg_debug_set_counter_wait_limit",
+           "dg_quantize_e4m3")
 
 
 class DgParams(ctypes.Structure):
@@ -20,7 +21,8 @@ class DgParams(ctypes.Structure):
                 ("hidden", ctypes.c_int), ("max_steps", ctypes.c_int), ("t_start", ctypes.c_float),
                 ("t_end", ctypes.c_float), ("eb_bound", ctypes.c_float), ("stop_thresh", ctypes.c_float),
                 ("stability", ctypes.c_int), ("tied", ctypes.c_int), ("group", ctypes.c_int),
-                ("accept_mode", ctypes.c_int), ("accept_rule", ctypes.c_int)]
+                ("accept_mode", ctypes.c_int), ("accept_rule", ctypes.c_int), ("logits_format", ctypes.c_int),
+                ("w_scale_exp", ctypes.c_int)]
 
 
 class DgError(RuntimeError):
@@ -74,6 +76,8 @@ def lib():
         L.dg_denoise_merge.restype = i32
         L.dg_debug_set_counter_wait_limit.argtypes = [ctypes.c_ulonglong]
         L.dg_debug_set_counter_wait_limit.restype = i32
+        L.dg_quantize_e4m3.argtypes = [vp, ctypes.c_longlong, i32, i32, vp, vp, vp]
+        L.dg_quantize_e4m3.restype = i32
         L.dg_profile_enable.argtypes = [i32]
         L.dg_profile_enable.restype = i32
         L.dg_profile_collect.argtypes = [ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_float),

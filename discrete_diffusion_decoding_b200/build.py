@@ -7,7 +7,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdg.so")
-SOURCES = ["dg_api.cu", "dg_fused.cu", "dg_small.cu", "dg_noalloc.cu"]
+SOURCES = ["dg_api.cu", "dg_fused.cu", "dg_small.cu", "dg_noalloc.cu", "dg_fp8.cu"]
 HEADERS = ["dg_common.cuh", "dg_fused.h", "dg_host.h", "dg_sm100.cuh", os.path.join("..", "..", "include", "dg.h")]
 
 

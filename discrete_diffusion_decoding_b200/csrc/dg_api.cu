@@ -1,6 +1,7 @@
 // C ABI of the denoise-sampling stage: argument checks, planning, workspace
 // layout, TMA descriptor encoding and the launch sequence of one step.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -57,11 +58,9 @@ bool current_device(int* dev) {
 // Caller holds g_dev_mu; `dev` is the current device.
 bool attr_set_locked(int dev) {
     if (g_attr_done[dev]) return true;
-    if (cudaFuncSetAttribute(dg_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(dg_fused_sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem) !=
-            cudaSuccess)
-        return false;
+    for (auto k : {dg_fused_kernel, dg_fused_sample_kernel, dg_fused_fp8_kernel, dg_fused_fp8_sample_kernel})
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem) != cudaSuccess)
+            return false;
     g_attr_done[dev] = true;
     return true;
 }
@@ -77,6 +76,7 @@ bool params_ok(const dg_params* p) {
     if (p->stability < 0) return false;
     if (p->accept_mode != 0 && p->accept_mode != 1) return false;
     if (p->accept_rule != 0 && p->accept_rule != 1) return false;
+    if (p->logits_format != 0 && p->logits_format != 1) return false;
     return true;
 }
 
@@ -111,6 +111,21 @@ bool encode_blocks_3d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t 
     cuuint32_t box[3] = {64, box_rows, box_blocks};
     cuuint32_t es[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The same view of a row-major matrix of 8-bit codes: {128 columns, rows, cols/128 blocks},
+// so a box of {128, box_rows, box_blocks} fills box_blocks 128-byte swizzle atoms.
+bool encode_bytes_3d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                     uint32_t box_blocks) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || cols % 128 != 0) return false;
+    cuuint64_t dims[3] = {128, rows, cols / 128};
+    cuuint64_t strides[2] = {cols, 128};
+    cuuint32_t box[3] = {128, box_rows, box_blocks};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -171,6 +186,7 @@ dg_status make_plan(const dg_params* p, int pairs, Plan* pl) {
     }
     const int G = p->hidden / slice;
     if (pairs < G) return DG_EUNSUPPORTED;
+    if (p->logits_format == 1 && p->hidden % 256 != 0) return DG_EUNSUPPORTED;   // 256 E4M3 values per stage
     Plan q{};
     q.C = p->n_canvas;
     q.N = p->n_canvas * kCanvas;
@@ -187,6 +203,7 @@ dg_status make_plan(const dg_params* p, int pairs, Plan* pl) {
         if (pg > q.max_seg) q.max_seg = pg;
     }
     q.n_slots = q.n_groups * q.max_seg;
+    q.fp8 = p->logits_format == 1;
     *pl = q;
     return DG_OK;
 }
@@ -223,8 +240,18 @@ dg_status launch_fused_and_combine(const dg_params* p, const Plan& pl, const Lay
     FusedArgs fa;
     std::memset(&fa, 0, sizeof(fa));
     const uint64_t prow_total = static_cast<uint64_t>(pl.n_groups) * 2 * pl.group * kCanvas;
-    if (!encode_blocks_3d(&fa.map_h, io.h, pl.N, pl.d, kTileM, kKChunk / 64) ||
-        !encode_blocks_3d(&fa.map_w, io.W, io.vocab_rows, pl.d, kBV / 2, kKChunk / 64) ||
+    if (pl.fp8) {
+        // the step's hidden states to E4M3 codes with a power-of-two scale per position
+        dg_quant_rows_kernel<<<pl.N, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(io.h), pl.d,
+                                                  at<uint8_t>(ws, L.hq), at<int32_t>(ws, L.hexp));
+        if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
+    }
+    const bool maps_ok =
+        pl.fp8 ? encode_bytes_3d(&fa.map_h, at<void>(ws, L.hq), pl.N, pl.d, kTileM, 2) &&
+                     encode_bytes_3d(&fa.map_w, io.W, io.vocab_rows, pl.d, kBV / 2, 2)
+               : encode_blocks_3d(&fa.map_h, io.h, pl.N, pl.d, kTileM, kKChunk / 64) &&
+                     encode_blocks_3d(&fa.map_w, io.W, io.vocab_rows, pl.d, kBV / 2, kKChunk / 64);
+    if (!maps_ok ||
         !encode_blocks_3d(&fa.map_e, io.E, io.vocab_rows, pl.d, kVChunk, pl.slice / 128) ||
         !encode_blocks_3d(&fa.map_p, at<void>(ws, L.pbuf), prow_total, kCanvas, kVChunk, 2))
         return DG_ECUDA;
@@ -246,7 +273,11 @@ dg_status launch_fused_and_combine(const dg_params* p, const Plan& pl, const Lay
     fa.vocab_offset = io.vocab_offset;
     fa.d = pl.d;
     fa.G = pl.group;
-    fa.keep_w_stages = io.E == io.W ? (pl.d / kKChunk) * kKeepWTenths / 10 : 0;
+    fa.keep_w_stages = (io.E == io.W && !pl.fp8) ? (pl.d / kKChunk) * kKeepWTenths / 10 : 0;
+    if (pl.fp8) {
+        fa.row_exp = at<int32_t>(ws, L.hexp);
+        fa.w_exp = p->w_scale_exp;
+    }
     fa.slice = pl.slice;
     fa.n_groups = pl.n_groups;
     fa.steps_per_tile = (io.vocab_rows + pl.group * kBV - 1) / (pl.group * kBV);
@@ -269,8 +300,9 @@ dg_status launch_fused_and_combine(const dg_params* p, const Plan& pl, const Lay
     cfg.numAttrs = 1;
     const bool prof = g_prof.on && g_prof.used < g_prof.max_records;
     if (prof && cudaEventRecord(g_prof.start[g_prof.used], s) != cudaSuccess) return DG_ECUDA;
-    if (cudaLaunchKernelEx(&cfg, p->accept_mode == 1 ? dg_fused_sample_kernel : dg_fused_kernel, fa) != cudaSuccess)
-        return DG_ECUDA;
+    void (*kern)(const FusedArgs) = p->accept_mode == 1 ? (pl.fp8 ? dg_fused_fp8_sample_kernel : dg_fused_sample_kernel)
+                                                        : (pl.fp8 ? dg_fused_fp8_kernel : dg_fused_kernel);
+    if (cudaLaunchKernelEx(&cfg, kern, fa) != cudaSuccess) return DG_ECUDA;
     if (prof) {
         if (cudaEventRecord(g_prof.stop[g_prof.used], s) != cudaSuccess) return DG_ECUDA;
         ++g_prof.used;
@@ -455,7 +487,7 @@ dg_status dg_denoise_step(const dg_params* p, int step, const void* h_dev, const
     if (r != DG_OK) return r;
     r = launch_stop(p, pl, L, workspace_dev, step, seeds_dev, tokens_dev, entropy_dev, argmax_dev, accept_dev, s);
     if (r != DG_OK) return r;
-    g_last_launches = 3;
+    g_last_launches = pl.fp8 ? 4 : 3;
     return DG_OK;
 }
 
@@ -474,6 +506,7 @@ dg_status dg_denoise_partial(const dg_params* p, int step, int v_begin, int v_co
     dg_status st = plan_current_device(p, &pl);
     if (st != DG_OK) return st;
     if (step < 1 || step > p->max_steps) return DG_EINVAL;
+    if (pl.fp8) return DG_EUNSUPPORTED;
     if (v_begin < 0 || v_count < kBV || v_begin % kBV != 0 || v_count % kBV != 0 ||
         static_cast<long long>(v_begin) + v_count > p->vocab)
         return DG_EINVAL;
@@ -505,6 +538,7 @@ dg_status dg_denoise_merge(const dg_params* p, int step, int n_parts, const void
     dg_status st = plan_current_device(p, &pl);
     if (st != DG_OK) return st;
     if (step < 1 || step > p->max_steps) return DG_EINVAL;
+    if (pl.fp8) return DG_EUNSUPPORTED;
     if (n_parts < 1 || n_parts > kMaxParts) return DG_EINVAL;
     if (!partials_dev || !seeds_dev || !tokens_dev || !entropy_dev || !argmax_dev || !accept_dev || !workspace_dev)
         return DG_EINVAL;
@@ -544,6 +578,35 @@ dg_status dg_denoise_merge(const dg_params* p, int step, int n_parts, const void
     st = launch_stop(p, pl, L, workspace_dev, step, seeds_dev, tokens_dev, entropy_dev, argmax_dev, accept_dev, s);
     if (st != DG_OK) return st;
     g_last_launches = 2;
+    return DG_OK;
+}
+
+dg_status dg_quantize_e4m3(const void* src_dev, long long rows, int cols, int per_row, uint8_t* codes_dev,
+                           int32_t* exps_dev, void* stream) {
+    g_last_launches = 0;
+    if (!src_dev || !codes_dev || !exps_dev || rows < 1 || cols < 2 || cols % 2 != 0) return DG_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(src_dev) | reinterpret_cast<uintptr_t>(codes_dev) |
+         reinterpret_cast<uintptr_t>(exps_dev)) & 3u)
+        return DG_EINVAL;
+    if (per_row && rows > 0x7fffffffLL) return DG_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(src_dev);
+    if (per_row) {
+        dg_quant_rows_kernel<<<static_cast<unsigned>(rows), 256, 0, s>>>(src, cols, codes_dev, exps_dev);
+        if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
+        g_last_launches = 1;
+        return DG_OK;
+    }
+    const long long n_pairs = rows * static_cast<long long>(cols) / 2;
+    long long blocks = (n_pairs + 255) / 256;
+    const long long cap = static_cast<long long>(device_sm_count()) * 8;
+    if (cap > 0 && blocks > cap) blocks = cap;
+    if (cudaMemsetAsync(exps_dev, 0, sizeof(int32_t), s) != cudaSuccess) return DG_ECUDA;
+    dg_amax_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(src, n_pairs, reinterpret_cast<uint32_t*>(exps_dev));
+    dg_amax_to_exp_kernel<<<1, 32, 0, s>>>(exps_dev);
+    dg_quant_tensor_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(src, n_pairs, codes_dev, exps_dev);
+    if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
+    g_last_launches = 3;
     return DG_OK;
 }
 

@@ -86,6 +86,7 @@ struct Plan {
     int steps_per_tile;  // vocabulary blocks of G * kBV rows per canvas
     int max_seg;      // partial slots per group
     int n_slots;      // n_groups * max_seg
+    int fp8;          // E4M3 logits operands (the workspace then holds the quantised hidden states)
 };
 
 struct Layout {
@@ -99,6 +100,7 @@ struct Layout {
     size_t sidx;                                  // [n_slots][G][256] int32: its vocabulary index
     size_t kept;                                  // [N] int32: token an accepted position keeps (group rule)
     size_t opart;                                 // [n_slots][256][d] float
+    size_t hq, hexp;                              // E4M3 logits: [N][d] codes and [N] exponents of h
     size_t total;
 };
 
@@ -125,6 +127,10 @@ inline Layout make_layout(const Plan& pl) {
     L.sidx = take(sizeof(int32_t) * static_cast<size_t>(pl.n_slots) * pl.group * kCanvas);
     L.kept = take(sizeof(int32_t) * pl.N);
     L.opart = take(sizeof(float) * static_cast<size_t>(pl.n_slots) * kCanvas * pl.d);
+    if (pl.fp8) {
+        L.hq = take(static_cast<size_t>(pl.N) * pl.d);
+        L.hexp = take(sizeof(int32_t) * static_cast<size_t>(pl.N));
+    }
     L.total = o;
     return L;
 }

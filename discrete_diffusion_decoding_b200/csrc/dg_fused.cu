@@ -172,7 +172,7 @@ __device__ __forceinline__ float neg_log2_uniform(uint32_t w) {
     return eps < 0.00390625f ? series : -fast_log2(1.0f - eps);
 }
 
-template <bool kSample>
+template <bool kSample, bool kFp8>
 __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* a_ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -245,6 +245,8 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
     uint32_t* cnt_rowmax = a.counters + counter_word(g, kCntRowmax);
     uint32_t* cnt_p = a.counters + counter_word(g, kCntP);
     uint32_t* cnt_used = a.counters + counter_word(g, kCntUsed);
+    // logits stages per W tile: 256 bytes of each row per stage (128 bf16 or 256 E4M3 values)
+    const int n_sstages = kFp8 ? a.d / 256 : a.d / kKChunk;
     const int n_ech = a.slice / 128;                 // E atoms (64 columns each) per CTA per O stage
     const uint32_t e_box_bytes = static_cast<uint32_t>(n_ech) * kAtomCol;   // <= kBox (slice <= 256)
     const int nG2 = 2 * G;                           // CTAs per group
@@ -280,7 +282,6 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 ++it;
                 return true;
             };
-            const int nkc = a.d / kKChunk;                 // logits stages per W tile
             auto emit_o = [&](int k, int t) -> bool {
                 if (a_side) {
                     if (!wait_counter(cnt_p, static_cast<uint32_t>(nG2 * (k + 1)), &abort_flag, a.err, kErrProducerP,
@@ -320,7 +321,7 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 for (int t = tb; t < te && ok; ++t, ++k) {
                     if (sub_valid(t, r)) {
                         const int v0 = vocab0(t, r) + static_cast<int>(prank) * (kBV / 2);
-                        for (int kc = 0; kc < nkc; ++kc) {
+                        for (int kc = 0; kc < n_sstages; ++kc) {
                             int slot;
                             if (!acquire(slot)) { ok = false; break; }
                             uint8_t* st = my_ring + slot * kBox;
@@ -356,7 +357,8 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
     } else if (warp == 1) {
         // ===================================================== pair UMMA issuer (leader CTA)
         if (lane == 0 && leader) {
-            const uint32_t idesc_s = idesc_bf16_f32(2 * kTileM, kBV, false, false);
+            const uint32_t idesc_s =
+                kFp8 ? idesc_e4m3_f32(2 * kTileM, kBV, false, false) : idesc_bf16_f32(2 * kTileM, kBV, false, false);
             const uint32_t idesc_o = idesc_bf16_f32(2 * kTileM, a.slice, true, true);
             uint32_t it = 0;
             bool ok = true;
@@ -413,16 +415,20 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                     }
                     tc_fence_after();
                     if (sub_valid(t, r)) {
-                        for (int kc = 0; kc < a.d / kKChunk; ++kc) {
+                        for (int kc = 0; kc < n_sstages; ++kc) {
                             uint32_t sta, stb;
                             if (!consume(sta, stb)) { ok = false; break; }
 #pragma unroll
-                            for (int kk = 0; kk < kKChunk / 16; ++kk) {
-                                // K step kk: atom column kk / 4, 32-byte offset (kk % 4) inside the swizzled row
+                            for (int kk = 0; kk < 8; ++kk) {
+                                // K step kk (32 bytes: 16 bf16 or 32 E4M3 values): atom column kk / 4,
+                                // 32-byte offset (kk % 4) inside the swizzled 128-byte row
                                 const uint32_t ko = (kk >> 2) * kAtomCol + (kk & 3) * 32;
                                 const uint64_t ad = smem_desc(sta + ko, 16, 1024, kSwizzle128B);
                                 const uint64_t bd = smem_desc(stb + ko, 16, 1024, kSwizzle128B);
-                                umma_ss_pair(tmem + kTmemS, ad, bd, idesc_s, (kc | kk) != 0 ? 1u : 0u);
+                                if constexpr (kFp8)
+                                    umma_ss_pair_f8(tmem + kTmemS, ad, bd, idesc_s, (kc | kk) != 0 ? 1u : 0u);
+                                else
+                                    umma_ss_pair(tmem + kTmemS, ad, bd, idesc_s, (kc | kk) != 0 ? 1u : 0u);
                             }
                             release();
                         }
@@ -455,7 +461,7 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
         const int crow = static_cast<int>(prank) * kTileM + row; // row within the canvas
         const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const bool sleader = (tid == kSoftmaxWarp0 * 32);
-        const float c2 = a.scale_log2;
+        float c2 = a.scale_log2;       // log2(e) / T times the row's operand scale (E4M3 logits)
         bool ok = true;
         int k = 0;
         for (int j = 0; j < sch.nseg && ok; ++j) {
@@ -463,6 +469,8 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
             if (!sch.seg(j, ct, tb, te)) continue;
             float m_ref = -INFINITY, l = 0.f, u = 0.f, best = -INFINITY;
             int best_idx = -1;
+            if constexpr (kFp8)
+                c2 = ldexpf(a.scale_log2, a.row_exp[active[ct] * kCanvas + crow] + a.w_exp);
             // sampled acceptance: Philox key of this canvas, counter word 3 of this position
             float skey = -INFINITY;
             int sidx = -1;
@@ -649,11 +657,19 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1) dg_fused_kernel(const __grid_constant__ FusedArgs a) {
-    fused_pass<false>(a);
+    fused_pass<false, false>(a);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) dg_fused_sample_kernel(const __grid_constant__ FusedArgs a) {
-    fused_pass<true>(a);
+    fused_pass<true, false>(a);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) dg_fused_fp8_kernel(const __grid_constant__ FusedArgs a) {
+    fused_pass<false, true>(a);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) dg_fused_fp8_sample_kernel(const __grid_constant__ FusedArgs a) {
+    fused_pass<true, true>(a);
 }
 
 // ---------------------------------------------------------------------------

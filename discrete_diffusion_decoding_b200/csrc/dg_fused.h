@@ -36,6 +36,10 @@ struct FusedArgs {
                          // tile keep normal L2 priority, so the self-conditioning pass finds them
                          // there (0 when E is a separate matrix)
     float scale_log2;    // log2(e) / T
+    // E4M3 logits (dg_fused_fp8_*): map_h / map_w view the 8-bit codes; row_exp [N] holds the hidden
+    // states' per-position exponents, w_exp the head's, so z = 2^(row_exp + w_exp) S / T
+    const int32_t* row_exp;
+    int w_exp;
     unsigned long long counter_wait_ns;   // limit of the waits on other CTAs' counters (the drains keep theirs)
 };
 
@@ -97,6 +101,14 @@ inline dim3 combine_grid(int N, int d) { return dim3(N, (d + kCombineCols - 1) /
 
 __global__ void dg_fused_kernel(const __grid_constant__ FusedArgs a);          // argmax acceptance
 __global__ void dg_fused_sample_kernel(const __grid_constant__ FusedArgs a);   // + Gumbel-max sample
+__global__ void dg_fused_fp8_kernel(const __grid_constant__ FusedArgs a);      // E4M3 logits operands
+__global__ void dg_fused_fp8_sample_kernel(const __grid_constant__ FusedArgs a);
+// E4M3 quantisation (dg_fp8.cu)
+__global__ void dg_quant_rows_kernel(const __nv_bfloat16* src, int cols, uint8_t* codes, int32_t* exps);
+__global__ void dg_amax_kernel(const __nv_bfloat16* src, long long n_pairs, uint32_t* amax_bits);
+__global__ void dg_amax_to_exp_kernel(int32_t* exps);
+__global__ void dg_quant_tensor_kernel(const __nv_bfloat16* src, long long n_pairs, uint8_t* codes,
+                                       const int32_t* exps);
 __global__ void dg_combine_kernel(const CombineArgs a);
 __global__ void dg_merge_kernel(const MergeArgs a);
 

@@ -75,6 +75,7 @@ extern "C" dg_status dg_denoise_stats_noalloc(const dg_params* p, int step, cons
     using namespace dg;
     host::set_last_launches(0);
     if (!p || step < 1 || step > p->max_steps) return DG_EINVAL;
+    if (p->logits_format != 0) return DG_EUNSUPPORTED;      // bf16 logits only
     if (!h_dev || !W_dev || !E_dev || !entropy_dev || !argmax_dev) return DG_EINVAL;
     const uintptr_t mis = reinterpret_cast<uintptr_t>(h_dev) | reinterpret_cast<uintptr_t>(W_dev) |
                           reinterpret_cast<uintptr_t>(E_dev) | reinterpret_cast<uintptr_t>(selfcond_dev);

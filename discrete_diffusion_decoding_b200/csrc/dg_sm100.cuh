@@ -319,6 +319,17 @@ __device__ __forceinline__ void umma_ss_pair(uint32_t d_tmem, uint64_t adesc, ui
         : "memory");
 }
 
+// The same pair UMMA on 8-bit operands (kind::f8f6f4; K = 32 per instruction, fp32 accumulation).
+__device__ __forceinline__ void umma_ss_pair_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+        : "memory");
+}
+
 // Arrive once on the barrier at this shared offset in every CTA of `mask` when all
 // pair UMMAs issued so far by this thread have completed.
 __device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
@@ -343,6 +354,12 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
     d |= static_cast<uint64_t>(1) << 46;
     d |= static_cast<uint64_t>(swizzle & 7u) << 61;
     return d;
+}
+
+// Instruction descriptor for kind::f8f6f4 with E4M3 A/B (format 0) and fp32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+    return (1u << 4) | (0u << 7) | (0u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.

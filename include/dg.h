@@ -108,6 +108,19 @@ typedef struct {
                          *       <= eb_bound - the sampler accepting token groups by entropy
                          *       (juhoplayground overview, entropy bounded sampler).  No position
                          *       is forced through.  Applied in the per-canvas stop kernel. */
+    int logits_format;  /* number format of the logits GEMM operands:
+                         *   0 = bf16 (default): W_dev holds the bf16 head;
+                         *   1 = E4M3: W_dev holds the head as 8-bit E4M3 codes [V, d] (one byte
+                         *       each, from dg_quantize_e4m3 with one scale for the tensor) whose
+                         *       values are decode(code) * 2^w_scale_exp; the hidden states are
+                         *       quantised per position to E4M3 with a power-of-two scale at every
+                         *       step, and z = 2^(e_h + w_scale_exp) (h_q . W_q) / T.  E_dev stays a
+                         *       bf16 embedding (for a tied head: the decoded codes, exact in bf16).
+                         *       Needs hidden a multiple of 256; dg_denoise_step only (the vocabulary
+                         *       split and the allocation-free entry point return DG_EUNSUPPORTED).
+                         *   The pages cite quantised deployments of the model (axbrief.com brief,
+                         *   GGUF sizes) but define no quantisation of this stage. */
+    int w_scale_exp;    /* logits_format 1: the power-of-two exponent of the head's scale */
 } dg_params;
 
 /* Fill a dg_params with the pages' defaults for C canvases of a (V, d) head. */
@@ -296,6 +309,21 @@ dg_status dg_denoise_merge(const dg_params* p, int step, int n_parts, const void
                            const uint64_t* seeds_dev, int32_t* tokens_dev, float* entropy_dev, int32_t* argmax_dev,
                            uint8_t* accept_dev, float* lse_dev, float* selfcond_dev, void* workspace_dev,
                            size_t workspace_bytes, void* stream);
+
+/*
+ * E4M3 quantisation (the 8-bit format of logits_format 1): sign bit, 4 exponent bits with
+ * bias 7, 3 mantissa bits, subnormals, largest finite value 448, no infinities.  Reads
+ * rows x cols bf16 values (row-major, src_dev), picks power-of-two scales 2^e - per row
+ * when per_row is 1 (exps_dev [rows] int32), else one for the whole tensor (exps_dev [1]) -
+ * with e the smallest integer such that every |x| 2^-e <= 448 (e = 0 for an all-zero row or
+ * tensor), and writes codes_dev [rows, cols] uint8 = x 2^-e rounded to the nearest E4M3 value,
+ * ties to the even mantissa (the scaling is exact, so only that rounding happens).
+ * cols must be even; all pointers 4-byte aligned.  Asynchronous on `stream`; the exponent
+ * stays on the device (copy exps_dev[0] to the host for dg_params.w_scale_exp).
+ * Errors: DG_EINVAL (null pointer, rows < 1, odd cols, misaligned), DG_ECUDA.
+ */
+dg_status dg_quantize_e4m3(const void* src_dev, long long rows, int cols, int per_row, uint8_t* codes_dev,
+                           int32_t* exps_dev, void* stream);
 
 /* Column-slice group size and group count the fused kernel uses for p on the current device. */
 dg_status dg_plan(const dg_params* p, int* group, int* n_groups, int* slice_cols);
