@@ -506,7 +506,6 @@ dg_status dg_denoise_partial(const dg_params* p, int step, int v_begin, int v_co
     dg_status st = plan_current_device(p, &pl);
     if (st != DG_OK) return st;
     if (step < 1 || step > p->max_steps) return DG_EINVAL;
-    if (pl.fp8) return DG_EUNSUPPORTED;
     if (v_begin < 0 || v_count < kBV || v_begin % kBV != 0 || v_count % kBV != 0 ||
         static_cast<long long>(v_begin) + v_count > p->vocab)
         return DG_EINVAL;
@@ -538,7 +537,6 @@ dg_status dg_denoise_merge(const dg_params* p, int step, int n_parts, const void
     dg_status st = plan_current_device(p, &pl);
     if (st != DG_OK) return st;
     if (step < 1 || step > p->max_steps) return DG_EINVAL;
-    if (pl.fp8) return DG_EUNSUPPORTED;
     if (n_parts < 1 || n_parts > kMaxParts) return DG_EINVAL;
     if (!partials_dev || !seeds_dev || !tokens_dev || !entropy_dev || !argmax_dev || !accept_dev || !workspace_dev)
         return DG_EINVAL;

@@ -116,8 +116,9 @@ typedef struct {
                          *       quantised per position to E4M3 with a power-of-two scale at every
                          *       step, and z = 2^(e_h + w_scale_exp) (h_q . W_q) / T.  E_dev stays a
                          *       bf16 embedding (for a tied head: the decoded codes, exact in bf16).
-                         *       Needs hidden a multiple of 256; dg_denoise_step only (the vocabulary
-                         *       split and the allocation-free entry point return DG_EUNSUPPORTED).
+                         *       Needs hidden a multiple of 256; dg_denoise_step and the vocabulary
+                         *       split (each shard's call passes the scale exponent of its own
+                         *       codes); the allocation-free entry point returns DG_EUNSUPPORTED.
                          *   The pages cite quantised deployments of the model (axbrief.com brief,
                          *   GGUF sizes) but define no quantisation of this stage. */
     int w_scale_exp;    /* logits_format 1: the power-of-two exponent of the head's scale */

@@ -126,15 +126,37 @@ def test_fp8_unsupported_shapes_and_paths(dg):
     with pytest.raises(_abi.DgError) as e:
         dg.dg_denoise_stats_noalloc(p, 1, x, x, x, x, x, None, None)
     assert e.value.status == _abi.DG_EUNSUPPORTED
-    ws = dg.Workspace(p)
-    part = torch.empty(dg.dg_partial_bytes(p), dtype=torch.uint8, device="cuda")
-    h = torch.zeros((256, 256), dtype=torch.bfloat16, device="cuda")
-    seeds = torch.zeros(1, dtype=torch.int64, device="cuda")
-    with pytest.raises(_abi.DgError) as e:
-        dg.dg_denoise_partial(p, 1, 0, 4096, h, h, h, seeds, part, ws)
-    assert e.value.status == _abi.DG_EUNSUPPORTED
     with pytest.raises(_abi.DgError) as e:
         dg.dg_quantize_e4m3(torch.zeros((4, 3), dtype=torch.bfloat16, device="cuda"),
                             torch.zeros((4, 3), dtype=torch.uint8, device="cuda"),
                             torch.zeros(4, dtype=torch.int32, device="cuda"), 1)            # odd column count
     assert e.value.status == _abi.DG_EINVAL
+
+
+def test_fp8_vocabulary_split_matches_single_call(dg):
+    """Two E4M3 shards (the head quantised once, its codes split by rows) merged equal the single
+    E4M3 call: the same logits, so the same argmax, accept flags and tokens."""
+    V, d, C = 4096, 512, 2
+    W = synth.weights(V, d, seed=1234)
+    codes, e, W64, E = _fp8_head(dg, W)
+    Ed = E.cuda()
+    h, _ = synth.spiked_hidden(W, C * 256, seed=66, gain_lo=0.5, gain_hi=30.0)
+    p = dg.params(C, V, d, logits_format=1, w_scale_exp=e, tied=0)
+    seeds = synth.canvas_seeds(C, base=710)
+    single = gc.gpu_step(dg, p, 3, h, codes, Ed, seeds)
+    ws, b = dg.Workspace(p), dg.StepBuffers(p)
+    seeds_t = torch.tensor(seeds.view(np.int64), device="cuda")
+    dg.dg_canvas_init(p, seeds_t, b.tokens, ws)
+    b.h.copy_(h.cuda())
+    nb = dg.dg_partial_bytes(p)
+    parts = torch.empty(2 * nb, dtype=torch.uint8, device="cuda")
+    for k, (v0, v1) in enumerate([(0, 1536), (1536, 4096)]):
+        dg.dg_denoise_partial(p, 3, v0, v1 - v0, b.h, codes[v0:v1], Ed[v0:v1], seeds_t, parts[k * nb:(k + 1) * nb], ws)
+    dg.dg_denoise_merge(p, 3, 2, parts, seeds_t, b.tokens, b.entropy, b.argmax, b.accept, b.lse, b.selfcond, ws)
+    dg.dg_stop_check(p, ws)
+    assert np.array_equal(b.argmax.cpu().numpy(), single["argmax"])
+    assert np.abs(b.entropy.cpu().numpy() - single["H"]).max() <= 1e-4
+    near = np.abs(single["H"] - p.eb_bound) < 1e-4
+    assert np.array_equal(b.accept.cpu().numpy()[~near], single["accept"][~near])
+    assert np.array_equal(b.tokens.cpu().numpy()[~near], single["tokens"][~near])
+    gc.report("fp8 vocabulary split 2 shards", C * 256, int(near.sum()))
