@@ -42,6 +42,7 @@ FLOPS_PER_STEP = 2 * (2.0 * N_POS * V * D)          # two contractions: logits a
 WE_BYTES_PER_STEP = 2.0 * V * D                     # tied bf16 W = E streamed once
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "dg_fused_kernel_single_step_v262144_d2816.md")
+PROFILE_SUMMARY_FP8 = os.path.join(ROOT, "profiles", "dg_fused_fp8_kernel_single_step_v262144_d2816.md")
 CSRC = os.path.join(ROOT, "discrete_diffusion_decoding_b200", "csrc")
 
 
@@ -107,10 +108,10 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def profiled_traffic():
+def profiled_traffic(path=None):
     """DRAM bytes per fused launch from the committed ncu summary, if it was taken on this kernel source."""
     try:
-        text = open(PROFILE_SUMMARY).read()
+        text = open(path or PROFILE_SUMMARY).read()
         src_hash = kernel_source_hash()
     except OSError:
         return None
@@ -164,11 +165,15 @@ class ClockSampler:
         self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
         self._stop = threading.Event()
 
+        def read():
+            self.rows.append((time.time(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                              nv.nvmlDeviceGetPowerUsage(h) / 1000.0, int(get_reasons(h))))
+        self._read = read
+
         def loop():
             while not self._stop.is_set():
                 try:
-                    self.rows.append((time.time(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
-                                      nv.nvmlDeviceGetPowerUsage(h) / 1000.0, int(get_reasons(h))))
+                    read()
                 except Exception as e:
                     self.err = str(e)
                     return
@@ -176,6 +181,20 @@ class ClockSampler:
         self._thread = threading.Thread(target=loop, daemon=True)
         self._thread.start()
         return self
+
+    def sample_now(self, n=3, gap_s=0.002):
+        """A few samples from the calling thread (while the GPU works through an enqueued region,
+        so that a short region is sampled even when the background thread does not get to run)."""
+        read = getattr(self, "_read", None)
+        if read is None:
+            return
+        for _ in range(n):
+            try:
+                read()
+            except Exception as e:
+                self.err = str(e)
+                return
+            time.sleep(gap_s)
 
     def __exit__(self, *exc):
         if self._thread is not None:
@@ -442,6 +461,7 @@ def run_gpu(args):
         for _ in range(args.steps):
             step()
         ev1.record(stream)
+        clk.sample_now()                 # the GPU is still working through the enqueued steps
         torch.cuda.synchronize()
         t_region1 = time.time()
     finally:
@@ -533,8 +553,8 @@ def run_gpu(args):
             bytes_launch = 3.0 * rows_per_rank * D
         roof_ms = max(flops_launch / (peak_tf * 1e12), bytes_launch / hbm) * 1e3
         # the committed DRAM capture is of the default kernel on the one-canvas tied workload
-        traffic = profiled_traffic() if (ACCEPT_MODE == 0 and CANVASES == 1 and not UNTIED and not split
-                                         and not LOGITS_FP8) else None
+        traffic = (profiled_traffic(PROFILE_SUMMARY_FP8 if LOGITS_FP8 else PROFILE_SUMMARY)
+                   if (ACCEPT_MODE == 0 and CANVASES == 1 and not UNTIED and not split) else None)
         positions = (1 if split else world) * N_POS
         value = positions / (ms_per_step * 1e-3)
         line = {
