@@ -298,6 +298,14 @@ def run_reference(args):
     h = synth.gaussian_hidden(N_POS, D, seed=42)
     W64, hb = stage.bf16_to_f64(synth.bf16_bits(W)), synth.bf16_bits(h)
     del W
+    if LOGITS_FP8:
+        # the E4M3 workload: the oracle decodes the quantised head and hidden states exactly
+        from oracle import fp8
+        codes, e = fp8.quantize_tensor(W64)
+        W64 = fp8.dequantize_tensor(codes, e)
+        del codes
+        hq, eh = fp8.quantize_rows(stage.bf16_to_f64(hb))
+        hb = stage.f64_to_bf16(fp8.dequantize_rows(hq, eh))
     T = stage.temperature(STEP, 48)
     _, probe_dt, _ = oracle_sample_rate(W64, hb, 8, T)
     full_est = probe_dt * N_POS / 8

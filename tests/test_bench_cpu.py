@@ -12,7 +12,7 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-@pytest.mark.parametrize("extra", [[], ["--accept", "sample"], ["--rule", "group"]])
+@pytest.mark.parametrize("extra", [[], ["--accept", "sample"], ["--rule", "group"], ["--logits", "e4m3"]])
 def test_reference_arm_json_line(extra):
     cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--vocab", "4096",
            "--steps", "2", "--warmup", "3"] + extra
@@ -30,6 +30,8 @@ def test_reference_arm_json_line(extra):
         assert "Gumbel-max" in d["config"]["workload"]
     if extra == ["--rule", "group"]:
         assert "cumulative entropy" in d["config"]["workload"]
+    if extra == ["--logits", "e4m3"]:
+        assert "E4M3" in d["config"]["workload"]
 
 
 def test_warmup_floor():
