@@ -182,6 +182,12 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
     // a_* / b_*: the A and B rings' barriers (full: the leader's, counting both CTAs' bytes)
     __shared__ uint64_t a_full[kAStages], a_empty[kAStages], b_full[kBStages], b_empty[kBStages];
     __shared__ uint64_t s_full, s_free, o_ready, o_done, drain_bar;
+    // producer drain: per side and ring slot, 1 + the index of the last use issued into it
+    // (0: none) and that use's bytes for one CTA (both CTAs load boxes of the same size);
+    // own_* this CTA's, peer_* (leader CTA) the peer's
+    __shared__ uint32_t own_use[2][kBStages], own_bytes[2][kBStages];
+    __shared__ uint32_t peer_use[2][kBStages], peer_bytes[2][kBStages];
+    __shared__ uint64_t peer_bar[2];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     __shared__ int n_active_s;
@@ -212,6 +218,12 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
         mbar_init(&o_ready, 2);              // leader: softmax of both CTAs
         mbar_init(&o_done, 1);
         mbar_init(&drain_bar, 1);
+        mbar_init(&peer_bar[0], 1);          // one remote arrival from the peer's producer of each side
+        mbar_init(&peer_bar[1], 1);
+        for (int i = 0; i < 2 * kBStages; ++i) {
+            own_use[i / kBStages][i % kBStages] = 0;
+            own_bytes[i / kBStages][i % kBStages] = 0;
+        }
         fence_mbar_init_cluster();
         abort_flag = 0;
         rescale_any = 0;
@@ -274,6 +286,9 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
             auto full_leader = [&](int slot) { return smem_addr_in_rank(&my_full[slot], 0); };
             uint32_t it = 0;
             bool ok = true;
+            const int side = a_side ? 0 : 1;
+            uint32_t* last_use = own_use[side];
+            uint32_t* last_bytes = own_bytes[side];
             auto acquire = [&](int& slot) -> bool {
                 slot = static_cast<int>(it % n_st);
                 if (it >= static_cast<uint32_t>(n_st) &&
@@ -281,6 +296,13 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                     return false;
                 ++it;
                 return true;
+            };
+            // a use of `slot` whose load brings `bytes` into each CTA of the pair; the leader
+            // posts both CTAs' bytes on its barrier
+            auto arm = [&](int slot, uint32_t bytes) {
+                last_use[slot] = it;
+                last_bytes[slot] = bytes;
+                if (leader) mbar_arrive_expect_tx(&my_full[slot], 2u * bytes);
             };
             auto emit_o = [&](int k, int t) -> bool {
                 if (a_side) {
@@ -298,12 +320,12 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                         if (!acquire(slot)) return false;
                         uint8_t* st = my_ring + slot * kBox;
                         if (a_side) {
-                            if (leader) mbar_arrive_expect_tx(&my_full[slot], 2u * 2u * kAtomCol);
+                            arm(slot, 2u * kAtomCol);
                             // both 64-row atoms of this CTA's canvas rows in one 3-D box
                             tma_load_3d_pair(st, &a.map_p, full_leader(slot), 0, prow + vc * kVChunk,
                                              static_cast<int>(prank) * 2);
                         } else {
-                            if (leader) mbar_arrive_expect_tx(&my_full[slot], 2u * e_box_bytes);
+                            arm(slot, e_box_bytes);
                             // this CTA's half of the column slice (n_ech atoms of 64 columns) in one 3-D box
                             tma_load_3d_pair_hint(st, &a.map_e, full_leader(slot), 0,
                                                   vocab0(t, q) + vc * kVChunk,
@@ -325,7 +347,7 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                             int slot;
                             if (!acquire(slot)) { ok = false; break; }
                             uint8_t* st = my_ring + slot * kBox;
-                            if (leader) mbar_arrive_expect_tx(&my_full[slot], 2u * kBox);
+                            arm(slot, kBox);
                             if (a_side) {
                                 tma_load_3d_pair(st, &a.map_h, full_leader(slot), 0, row0, kc * (kKChunk / 64));
                             } else {
@@ -341,15 +363,42 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 }
                 if (ok) ok = emit_o(k - 1, te - 1);
             }
-            // drain: every issued use of a stage has been released by the leader's
-            // commit, so no load into this CTA is still in flight when it exits
-            for (uint32_t u = (it > static_cast<uint32_t>(n_st) ? it - n_st : 0); u < it; ++u) {
-                const int slot = static_cast<int>(u % n_st);
-                const uint64_t t0 = global_ns();
-                while (!mbar_try_wait(smem_u32(&my_empty[slot]), (u / n_st) & 1)) {
-                    if (global_ns() - t0 > DG_WAIT_LIMIT_NS) {
-                        atomicCAS(a.err, 0, kErrProducerDrain);
-                        break;
+            // drain: every load issued into either CTA of the pair has landed before the
+            // pair passes its last cluster barrier.  All loads complete on the leader's full
+            // barriers, so the peer hands its last use of every slot to the leader, and the
+            // leader waits for the last phase of every slot.  A producer issues use u + n_st
+            // of a slot only after use u was consumed, which needs both CTAs' bytes; so after
+            // an abort the two CTAs' last uses of a slot differ by at most one round, and the
+            // leader settles that round: bytes the peer never sent are completed here, and a
+            // use only the peer issued is armed here with the peer's bytes.
+            if (!leader) {
+                for (int sl = 0; sl < n_st; ++sl) {
+                    st_shared_rank_u32(&peer_use[side][sl], 0, last_use[sl]);
+                    st_shared_rank_u32(&peer_bytes[side][sl], 0, last_bytes[sl]);
+                }
+                mbar_arrive_remote(&peer_bar[side], 0);      // release: the stores above first
+            } else {
+                auto drain_wait = [&](uint64_t* bar, uint32_t parity, bool cluster) -> bool {
+                    const uint32_t ba = smem_u32(bar);
+                    const uint64_t t0 = global_ns();
+                    while (!(cluster ? mbar_try_wait_cluster(ba, parity) : mbar_try_wait(ba, parity))) {
+                        if (global_ns() - t0 > DG_WAIT_LIMIT_NS) {
+                            atomicCAS(a.err, 0, kErrProducerDrain);
+                            return false;
+                        }
+                    }
+                    return true;
+                };
+                if (drain_wait(&peer_bar[side], 0, true)) {
+                    for (int sl = 0; sl < n_st; ++sl) {
+                        const uint32_t ul = last_use[sl], un = peer_use[side][sl];
+                        if (ul == 0 && un == 0) continue;
+                        if (ul > un)
+                            mbar_complete_tx(&my_full[sl], last_bytes[sl]);
+                        else if (un > ul)
+                            mbar_arrive_expect_tx(&my_full[sl], peer_bytes[side][sl]);
+                        const uint32_t u = (ul > un ? ul : un) - 1;
+                        if (!drain_wait(&my_full[sl], (u / n_st) & 1, false)) break;
                     }
                 }
             }

@@ -118,6 +118,20 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
     return ok != 0;
 }
 
+// Transaction bytes counted on a local barrier without a copy: stands in for bytes that
+// were expected but will never be sent (the drain of an aborted pass).
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+// Store to the same shared-memory variable in CTA `rank` of this cluster (made visible to
+// that CTA by a later release at cluster scope, e.g. mbar_arrive_remote).
+__device__ __forceinline__ void st_shared_rank_u32(uint32_t* p, uint32_t rank, uint32_t v) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(p)), "r"(rank));
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
+}
+
 // Raise the abort flag of this CTA and of the other CTA of its pair (same shared-memory
 // offset in cluster rank ctarank ^ 1): both CTAs then leave their loops together.  Only
 // valid in a kernel of 2-CTA clusters, between its first and last cluster barrier.
