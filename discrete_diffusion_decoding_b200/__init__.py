@@ -17,7 +17,7 @@ __all__ = ["DgError", "DgParams", "params", "workspace_size", "plan", "temperatu
            "dg_denoise_step", "dg_stop_check", "dg_stub_hidden", "last_launch_count", "profile_enable",
            "profile_collect", "dg_denoise_stats_noalloc", "dg_debug_set_error", "Workspace", "StepBuffers",
            "decode_batch", "decode_block_ar", "dg_partial_bytes", "dg_denoise_partial", "dg_denoise_merge",
-           "dg_debug_set_counter_wait_limit", "dg_quantize_e4m3", "quantize_head_e4m3"]
+           "dg_debug_set_counter_wait_limit", "dg_quantize_e4m3", "quantize_head_e4m3", "dg_last_sm_clock"]
 
 
 def params(n_canvas, vocab, hidden, **overrides):
@@ -132,6 +132,15 @@ def quantize_head_e4m3(W, stream=None):
     exps = torch.empty(1, dtype=torch.int32, device=W.device)
     dg_quantize_e4m3(W, codes, exps, 0, stream)
     return codes, int(exps.item())
+
+
+def dg_last_sm_clock(p, ws, stream=None):
+    """SM clock (MHz) at which the last fused pass on this workspace issued its tensor-core work
+    (0.0 before the first pass after dg_canvas_init); synchronises the stream."""
+    mhz = ctypes.c_float()
+    check("dg_last_sm_clock", lib().dg_last_sm_clock(ctypes.byref(p), ws.ptr, ws.nbytes, ctypes.byref(mhz),
+                                                     _stream(stream)))
+    return float(mhz.value)
 
 
 def dg_debug_set_counter_wait_limit(ns):

@@ -13,7 +13,7 @@ EXPORTS = ("dg_params_default", "dg_temperature", "dg_workspace_size", "dg_canva
            "dg_stop_check", "dg_stub_hidden", "dg_status_string", "dg_last_launch_count", "dg_plan",
            "dg_profile_enable", "dg_profile_collect", "dg_denoise_stats_noalloc", "dg_debug_set_error",
            "dg_partial_bytes", "dg_denoise_partial", "dg_denoise_merge", "dg_debug_set_counter_wait_limit",
-           "dg_quantize_e4m3")
+           "dg_quantize_e4m3", "dg_last_sm_clock")
 
 
 class DgParams(ctypes.Structure):
@@ -78,6 +78,8 @@ def lib():
         L.dg_debug_set_counter_wait_limit.restype = i32
         L.dg_quantize_e4m3.argtypes = [vp, ctypes.c_longlong, i32, i32, vp, vp, vp]
         L.dg_quantize_e4m3.restype = i32
+        L.dg_last_sm_clock.argtypes = [P, vp, sz, ctypes.POINTER(ctypes.c_float), vp]
+        L.dg_last_sm_clock.restype = i32
         L.dg_profile_enable.argtypes = [i32]
         L.dg_profile_enable.restype = i32
         L.dg_profile_collect.argtypes = [ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_float),

@@ -264,6 +264,7 @@ dg_status launch_fused_and_combine(const dg_params* p, const Plan& pl, const Lay
     fa.stat_idx = at<int32_t>(ws, L.stat_idx);
     fa.opart = at<float>(ws, L.opart);
     fa.err = at<int>(ws, L.err);
+    fa.clk = at<unsigned long long>(ws, L.clk);
     fa.seeds = io.seeds;
     fa.skey = at<float>(ws, L.skey);
     fa.sidx = at<int32_t>(ws, L.sidx);
@@ -445,7 +446,9 @@ dg_status dg_canvas_init(const dg_params* p, const uint64_t* seeds_dev, int32_t*
     const int blocks = (pl.N + threads - 1) / threads;
     dg_init_kernel<<<blocks, threads, 0, s>>>(seeds_dev, tokens_dev, at<int32_t>(workspace_dev, L.prev_argmax),
                                               at<int32_t>(workspace_dev, L.stable), at<int32_t>(workspace_dev, L.stop),
-                                              at<int32_t>(workspace_dev, L.err), at<uint32_t>(workspace_dev, L.counters),
+                                              at<int32_t>(workspace_dev, L.err),
+                                              at<unsigned long long>(workspace_dev, L.clk),
+                                              at<uint32_t>(workspace_dev, L.counters),
                                               pl.n_groups * 128, pl.C, pl.V);
     if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
     g_last_launches = 1;
@@ -682,6 +685,26 @@ dg_status dg_stop_check(const dg_params* p, void* workspace_dev, size_t workspac
         *n_stopped_host = n;
     }
     if (err_word != 0) return DG_ETIMEOUT;
+    return DG_OK;
+}
+
+dg_status dg_last_sm_clock(const dg_params* p, const void* workspace_dev, size_t workspace_bytes, float* mhz_host,
+                           void* stream) {
+    if (!workspace_dev || !mhz_host) return DG_EINVAL;
+    Plan pl;
+    const dg_status st = plan_current_device(p, &pl);
+    if (st != DG_OK) return st;
+    const Layout L = make_layout(pl);
+    if (workspace_bytes < L.total) return DG_ENOMEM;
+    unsigned long long v[4] = {0, 0, 0, 0};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(v, static_cast<const uint8_t*>(workspace_dev) + L.clk, sizeof(v), cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return DG_ECUDA;
+    *mhz_host = (v[3] > v[1] && v[2] > v[0])
+                    ? static_cast<float>(static_cast<double>(v[2] - v[0]) / static_cast<double>(v[3] - v[1]) * 1e3)
+                    : 0.f;
     return DG_OK;
 }
 

@@ -91,6 +91,8 @@ struct Plan {
 
 struct Layout {
     size_t prev_argmax, stable, stop, err;        // per-canvas state
+    size_t clk;                                   // [4] uint64: SM cycles and global ns at the start
+                                                  // and end of CTA 0's MMA loop (last fused pass)
     size_t counters;                              // [n_groups][4] uint32, 128 B apart
     size_t rowmax;                                // [n_groups][2][G][256] float
     size_t pbuf;                                  // [n_groups][2][G][kBV vocab][256 rows] bf16 (P^T)
@@ -118,6 +120,7 @@ inline Layout make_layout(const Plan& pl) {
     L.stable = take(sizeof(int32_t) * pl.C);
     L.stop = take(sizeof(int32_t) * pl.C);
     L.err = take(sizeof(int32_t) * 4);
+    L.clk = take(sizeof(unsigned long long) * 4);
     L.counters = take(static_cast<size_t>(128) * 4 * pl.n_groups);
     L.rowmax = take(sizeof(float) * pl.n_groups * 2 * pl.group * kCanvas);
     L.pbuf = take(static_cast<size_t>(2) * pl.n_groups * 2 * pl.group * kCanvas * kBV);

@@ -454,6 +454,8 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                 return true;
             };
             int k = 0;
+            // the SM clock this pass runs at: cycles and global time over CTA 0's issue loop
+            const unsigned long long clk0 = clock64(), ns0 = global_ns();
             for (int j = 0; j < sch.nseg && ok; ++j) {
                 int ct, tb, te;
                 if (!sch.seg(j, ct, tb, te)) continue;
@@ -490,6 +492,13 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                     if (t > tb) ok = do_o(k - 1, t - 1, t - 1 == tb);
                 }
                 if (ok) ok = do_o(k - 1, te - 1, te - 1 == tb);
+            }
+            if (blockIdx.x == 0) {
+                const unsigned long long clk1 = clock64(), ns1 = global_ns();
+                a.clk[0] = clk0;
+                a.clk[1] = ns0;
+                a.clk[2] = clk1;
+                a.clk[3] = ns1;
             }
             // drain: all issued UMMAs complete before TMEM is released
             umma_commit_pair(&drain_bar, 0x1);

@@ -23,6 +23,7 @@ struct FusedArgs {
     int32_t* stat_idx;
     float* opart;
     int* err;
+    unsigned long long* clk;   // CTA 0 writes SM cycles and global ns at the start and end of its MMA loop
     // sampled acceptance (dg_fused_sample_kernel only): per-canvas Philox seeds, the
     // step, and the best Gumbel-max key / index of every (piece, pair, position)
     const uint64_t* seeds;
@@ -114,7 +115,8 @@ __global__ void dg_merge_kernel(const MergeArgs a);
 
 // small kernels (dg_small.cu)
 __global__ void dg_init_kernel(const uint64_t* seeds, int32_t* tokens, int32_t* prev_argmax, int32_t* stable,
-                               int32_t* stop, int32_t* err, uint32_t* counters, int n_counter_words, int C, int V);
+                               int32_t* stop, int32_t* err, unsigned long long* clk, uint32_t* counters,
+                               int n_counter_words, int C, int V);
 // Group entropy-bounded accept, applied by dg_stop_kernel before the stop reduction
 // when `rule` is 1 (nothing happens with rule 0 or a null tokens pointer).
 struct GroupAcceptArgs {

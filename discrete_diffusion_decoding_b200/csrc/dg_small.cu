@@ -13,7 +13,8 @@ namespace dg {
 // juhoplayground, entropy bounded sampler: start from uniform random tokens),
 // plus a reset of the per-canvas state.
 __global__ void dg_init_kernel(const uint64_t* seeds, int32_t* tokens, int32_t* prev_argmax, int32_t* stable,
-                               int32_t* stop, int32_t* err, uint32_t* counters, int n_counter_words, int C, int V) {
+                               int32_t* stop, int32_t* err, unsigned long long* clk, uint32_t* counters,
+                               int n_counter_words, int C, int V) {
     const int n = blockIdx.x * blockDim.x + threadIdx.x;
     const int N = C * kCanvas;
     if (n < N) {
@@ -26,7 +27,10 @@ __global__ void dg_init_kernel(const uint64_t* seeds, int32_t* tokens, int32_t* 
         stable[n] = 0;
         stop[n] = 0;
     }
-    if (n < 4) err[n] = 0;
+    if (n < 4) {
+        err[n] = 0;
+        clk[n] = 0ull;
+    }
     for (int w = n; w < n_counter_words; w += gridDim.x * blockDim.x) counters[w] = 0u;
 }
 

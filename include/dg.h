@@ -184,6 +184,19 @@ dg_status dg_stop_check(const dg_params* p, void* workspace_dev, size_t workspac
                         int32_t* stable_host, int* n_stopped_host, void* stream);
 
 /*
+ * Telemetry (not on the pages): the SM clock, in MHz, at which the last fused pass run with
+ * this workspace issued its tensor-core work - CTA 0's cycle counter over the global timer
+ * across its issue loop (the same interval on both).  The clock a dense tensor-core pass
+ * actually runs at sits below the one the driver reports when power limits it, and it
+ * sets the pass's time; reading it explains a roofline fraction.  Copies 32 bytes from the
+ * workspace and synchronises `stream`; *mhz_host = 0 when no pass has run since
+ * dg_canvas_init.  Errors: DG_EINVAL (null pointer), DG_ENOMEM (workspace too small for
+ * p), DG_ECUDA.
+ */
+dg_status dg_last_sm_clock(const dg_params* p, const void* workspace_dev, size_t workspace_bytes, float* mhz_host,
+                           void* stream);
+
+/*
  * Host-side fault injection for the error path (not on the pages): writes `code`
  * into the workspace's device error word, stream-ordered, exactly as a bounded
  * in-kernel wait that runs out would.  The next dg_stop_check then reports

@@ -63,3 +63,15 @@ def test_sm100a_only_build():
     from discrete_diffusion_decoding_b200 import build
     src = open(build.__file__).read()
     assert "arch=compute_100a,code=sm_100a" in src
+
+
+def test_last_sm_clock_argument_checks_without_device(lib):
+    from discrete_diffusion_decoding_b200 import _abi
+    p = _abi.DgParams()
+    lib.dg_params_default(ctypes.byref(p), 1, 4096, 512)
+    lib.dg_last_sm_clock.argtypes = [ctypes.POINTER(_abi.DgParams), ctypes.c_void_p, ctypes.c_size_t,
+                                     ctypes.POINTER(ctypes.c_float), ctypes.c_void_p]
+    lib.dg_last_sm_clock.restype = ctypes.c_int
+    mhz = ctypes.c_float()
+    assert lib.dg_last_sm_clock(ctypes.byref(p), None, 1 << 20, ctypes.byref(mhz), None) == _abi.DG_EINVAL
+    assert lib.dg_last_sm_clock(ctypes.byref(p), 1 << 20, 1 << 20, None, None) == _abi.DG_EINVAL

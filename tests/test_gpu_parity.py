@@ -4,6 +4,7 @@ Every test here runs the library's sm_100a kernels on a B200 and compares with
 the oracle on the same seeded inputs (see gpu_case.py for the tolerances).
 """
 
+import ctypes
 import math
 
 import numpy as np
@@ -381,6 +382,34 @@ def test_forced_error_word_reported_and_cleared(dg):
     with pytest.raises(_abi.DgError) as e:
         dg.dg_debug_set_error(p, small, 1)
     assert e.value.status == _abi.DG_ENOMEM
+
+
+def test_last_sm_clock_telemetry(dg):
+    """dg_last_sm_clock: 0 after dg_canvas_init, then the clock of the last fused pass, a value
+    between the lowest and highest SM clocks a B200 runs at; argument errors are reported."""
+    from discrete_diffusion_decoding_b200 import _abi
+    V, d = 65536, 512
+    p = dg.params(1, V, d)
+    ws, bufs = dg.Workspace(p), dg.StepBuffers(p)
+    W = synth.weights(V, d).cuda()
+    seeds = torch.zeros(1, dtype=torch.int64, device="cuda")
+    dg.dg_canvas_init(p, seeds, bufs.tokens, ws)
+    assert dg.dg_last_sm_clock(p, ws) == 0.0
+    bufs.h.copy_(synth.gaussian_hidden(256, d).cuda())
+    dg.dg_denoise_step(p, 1, bufs.h, W, W, seeds, bufs.tokens, bufs.entropy, bufs.argmax, bufs.accept, bufs.lse,
+                       bufs.selfcond, ws)
+    mhz = dg.dg_last_sm_clock(p, ws)
+    assert 300.0 < mhz < 2200.0, mhz
+    dg.dg_canvas_init(p, seeds, bufs.tokens, ws)
+    assert dg.dg_last_sm_clock(p, ws) == 0.0
+    small = dg.Workspace(p)
+    small.nbytes = 64
+    with pytest.raises(_abi.DgError) as e:
+        dg.dg_last_sm_clock(p, small)
+    assert e.value.status == _abi.DG_ENOMEM
+    mhz_c = ctypes.c_float()
+    assert dg.lib().dg_last_sm_clock(ctypes.byref(p), None, ws.nbytes, ctypes.byref(mhz_c), None) == _abi.DG_EINVAL
+    assert dg.lib().dg_last_sm_clock(ctypes.byref(p), ws.ptr, ws.nbytes, None, None) == _abi.DG_EINVAL
 
 
 def test_all_canvases_stopped_step_is_a_no_op(dg):
