@@ -36,12 +36,14 @@
 //    come from DRAM once and are shared through L2); each piece ends with O and
 //    the statistics written as a partial, merged by dg_combine_kernel.
 //
-// Roles inside a CTA (256 threads): warps 0 and 3 issue TMA loads (A and B
-// operands) into a 3-stage ring of 64 KB stages (both CTAs of a pair load;
-// completion is counted on the leader's barriers); warp 1 allocates TMEM and,
-// in the leader CTA, issues the pair UMMAs; warps 4-7 (one TMEM lane quarter
-// each, thread = position row) do the softmax, publish P^T and run the epilogue.
-// Every wait is bounded (see dg_sm100.cuh).
+// Roles inside a CTA (256 threads): warp 0 issues the A operand's TMA loads
+// (h, or P^T) into a ring of 3 x 32 KB stages and warp 3 the B operand's (W, or
+// E) into a ring of 4 x 32 KB stages (both CTAs of a pair load; completion is
+// counted on the leader's barriers); warp 1 allocates TMEM and, in the leader
+// CTA, issues the pair UMMAs; warps 4-7 (one TMEM lane quarter each, thread =
+// position row) do the softmax, publish P^T and run the epilogue.  Every wait is
+// bounded (see dg_sm100.cuh); the producers leave only once every load they
+// issued into either CTA has landed.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
