@@ -113,6 +113,46 @@ def test_step_groups_and_segments(dg, group, tied, C, V, d):
     gc.compare(g, o, _rows_all(C * 256), p.eb_bound, tag=f"G={group}")
 
 
+def _widest_hidden(dg, V):
+    """The widest hidden size whose group (one pair per 256 columns) still fits on the device at once."""
+    from discrete_diffusion_decoding_b200 import _abi
+    for k in range(96, 0, -1):
+        try:
+            pl = dg.plan(dg.params(1, V, 256 * k))
+        except _abi.DgError as e:
+            assert e.status == _abi.DG_EUNSUPPORTED
+            continue
+        return 256 * k, pl
+    raise AssertionError("no hidden size fits")
+
+
+@pytest.mark.parametrize("which", ["d5376", "widest"])
+def test_wide_hidden_groups(dg, which):
+    """Wide hidden sizes: 21-pair groups (d = 5376, three groups), and the widest group the device holds
+    at once (one group of every resident pair, a single ragged vocabulary block), on every row."""
+    from discrete_diffusion_decoding_b200 import _abi
+    if which == "d5376":
+        V, d = 16384, 5376
+        pl = dg.plan(dg.params(1, V, d))
+        assert pl["group"] == 21 and pl["slice"] == 256
+    else:
+        V = 4096
+        d, pl = _widest_hidden(dg, V)
+        assert pl["n_groups"] == 1 and pl["group"] == d // 256 >= 64
+        with pytest.raises(_abi.DgError) as e:                  # one more pair than fits
+            dg.plan(dg.params(1, V, d + 256))
+        assert e.value.status == _abi.DG_EUNSUPPORTED
+    W = synth.weights(V, d, seed=71)
+    h, _ = synth.spiked_hidden(W, 256, seed=72, gain_lo=0.5, gain_hi=30.0)
+    p = dg.params(1, V, d)
+    seeds = synth.canvas_seeds(1, base=300)
+    Wd = W.cuda()
+    g = gc.gpu_step(dg, p, 2, h, Wd, Wd, seeds)
+    o = gc.oracle_rows(gc.bits(h), gc.bits(W), gc.bits(W), dg.temperature(p, 2), p.eb_bound, seeds, 2,
+                       _rows_all(256), V)
+    gc.compare(g, o, _rows_all(256), p.eb_bound, tag=f"d={d} G={pl['group']} groups={pl['n_groups']}")
+
+
 def test_large_logits_rescale(dg):
     """Rows whose running maximum jumps late in the vocabulary force the lazy rescale of O."""
     V, d, C = 131072, 512, 1          # G = 2: 256 blocks per tile, several blocks per segment
