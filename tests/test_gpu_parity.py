@@ -113,6 +113,25 @@ def test_step_groups_and_segments(dg, group, tied, C, V, d):
     gc.compare(g, o, _rows_all(C * 256), p.eb_bound, tag=f"G={group}")
 
 
+@pytest.mark.parametrize("C,mode", [(1, 0), (5, 0), (5, 1)])
+def test_smallest_shape(dg, C, mode):
+    """The smallest accepted head (V = 256: one vocabulary tile; d = 128: one 128-column stage and
+    slice) with one and several canvases, argmax and sampled acceptance, on every row."""
+    V, d = 256, 128
+    W = synth.weights(V, d, seed=81)
+    h, _ = synth.spiked_hidden(W, C * 256, seed=82, gain_lo=0.5, gain_hi=60.0)
+    p = dg.params(C, V, d, accept_mode=mode, eb_bound=4.0 if mode else 0.1)
+    assert dg.plan(p)["group"] == 1
+    seeds = synth.canvas_seeds(C, base=400)
+    Wd = W.cuda()
+    g = gc.gpu_step(dg, p, 1, h, Wd, Wd, seeds)
+    o = gc.oracle_rows(gc.bits(h), gc.bits(W), gc.bits(W), dg.temperature(p, 1), p.eb_bound, seeds, 1,
+                       _rows_all(C * 256), V, accept_mode=mode)
+    excl, _, _ = gc.compare(g, o, _rows_all(C * 256), p.eb_bound, tag=f"V=256 d=128 C={C} mode={mode}")
+    assert len(excl) < C * 256 // 4
+    assert int(g["accept"].sum()) > 0
+
+
 def _widest_hidden(dg, V):
     """The widest hidden size whose group (one pair per 256 columns) still fits on the device at once."""
     from discrete_diffusion_decoding_b200 import _abi
