@@ -75,3 +75,29 @@ def test_last_sm_clock_argument_checks_without_device(lib):
     mhz = ctypes.c_float()
     assert lib.dg_last_sm_clock(ctypes.byref(p), None, 1 << 20, ctypes.byref(mhz), None) == _abi.DG_EINVAL
     assert lib.dg_last_sm_clock(ctypes.byref(p), 1 << 20, 1 << 20, None, None) == _abi.DG_EINVAL
+
+
+def test_defaults_match_the_pages_settings_table(lib):
+    """dg_params_default and the oracle's defaults carry the settings the pages print
+    (tests/golden/sampler_settings.txt)."""
+    import inspect
+
+    from discrete_diffusion_decoding_b200 import _abi
+    from oracle import decode, stage
+    want = {}
+    for line in open(os.path.join(ROOT, "tests", "golden", "sampler_settings.txt")):
+        line = line.strip()
+        if line and not line.startswith("#"):
+            k, v = line.split()
+            want[k] = float(v)
+    p = _abi.DgParams()
+    lib.dg_params_default(ctypes.byref(p), 1, 4096, 128)
+    for k, v in want.items():
+        assert abs(getattr(p, k) - v) <= 1e-7 * max(1.0, v), k
+    sig = inspect.signature(decode.decode_batch).parameters
+    assert sig["max_steps"].default == want["max_steps"] and sig["t_start"].default == want["t_start"]
+    assert sig["t_end"].default == want["t_end"] and sig["bound"].default == want["eb_bound"]
+    assert sig["stop_thresh"].default == want["stop_thresh"] and sig["stability"].default == want["stability"]
+    # the schedule's end points (the oracle returns T in float32, the precision the kernel takes)
+    assert abs(stage.temperature(1, 48) - want["t_start"]) <= 1e-7
+    assert abs(stage.temperature(48, 48) - want["t_end"]) <= 1e-7
