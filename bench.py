@@ -493,10 +493,8 @@ def run_gpu(args):
     # neighbouring steps' compute; the small per-position results (which the next step
     # overwrites) are read back on the compute stream before it continues.
     h_pin = h_host.pin_memory()
-    out_H = torch.empty(N_POS, dtype=torch.float32).pin_memory()
-    out_tok = torch.empty(N_POS, dtype=torch.int32).pin_memory()
-    out_am = torch.empty(N_POS, dtype=torch.int32).pin_memory()
-    out_acc = torch.empty(N_POS, dtype=torch.uint8).pin_memory()
+    # entropy, tokens, argmax and accept flags in one pinned buffer (StepBuffers.packed)
+    out_small = torch.empty(bufs.packed.numel(), dtype=torch.uint8).pin_memory()
     out_sc = [torch.empty((N_POS, D), dtype=torch.float32).pin_memory() for _ in range(2)]
     e2e_steps = args.steps            # as long as the device-timed loop: the same clock regime
     copy_stream = torch.cuda.Stream(device=dev)
@@ -516,10 +514,7 @@ def run_gpu(args):
             stream.wait_event(h_ready[b])
             step(h_dev[b], sc_dev[b])
             with torch.cuda.stream(stream):
-                out_H.copy_(bufs.entropy, non_blocking=True)
-                out_tok.copy_(bufs.tokens, non_blocking=True)
-                out_am.copy_(bufs.argmax, non_blocking=True)
-                out_acc.copy_(bufs.accept, non_blocking=True)
+                out_small.copy_(bufs.packed, non_blocking=True)      # one copy for the per-position results
             done[b].record(stream)
             with torch.cuda.stream(copy_stream):
                 if i + 1 < n:
@@ -542,7 +537,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev if world > 1 else None) / e2e_steps
     h2d = h_pin.numel() * h_pin.element_size()
-    d2h = sum(t.numel() * t.element_size() for t in (out_H, out_tok, out_am, out_acc, out_sc[0]))
+    d2h = sum(t.numel() * t.element_size() for t in (out_small, out_sc[0]))
 
     line = None
     if rank == 0:

@@ -185,14 +185,20 @@ def dg_stub_hidden(p, step, gain, noise, seeds, E, tokens, h, ws, stream=None):
 
 
 class StepBuffers:
-    """Per-step outputs for N positions (device tensors)."""
+    """Per-step outputs for N positions (device tensors).
+
+    The per-position results a caller reads every step share one allocation, `packed`
+    (entropy float32 [N] | tokens int32 [N] | argmax int32 [N] | accept uint8 [N], 13 N
+    bytes), so one device-to-host copy returns them all; the named tensors are views of it.
+    """
 
     def __init__(self, p, device="cuda", selfcond=True):
         N, d = p.n_canvas * p.canvas_len, p.hidden
-        self.tokens = torch.empty(N, dtype=torch.int32, device=device)
-        self.entropy = torch.empty(N, dtype=torch.float32, device=device)
-        self.argmax = torch.empty(N, dtype=torch.int32, device=device)
-        self.accept = torch.empty(N, dtype=torch.uint8, device=device)
+        self.packed = torch.empty(13 * N, dtype=torch.uint8, device=device)
+        self.entropy = self.packed[0:4 * N].view(torch.float32)
+        self.tokens = self.packed[4 * N:8 * N].view(torch.int32)
+        self.argmax = self.packed[8 * N:12 * N].view(torch.int32)
+        self.accept = self.packed[12 * N:13 * N]
         self.lse = torch.empty(N, dtype=torch.float32, device=device)
         self.selfcond = torch.empty((N, d), dtype=torch.float32, device=device) if selfcond else None
         self.h = torch.empty((N, d), dtype=torch.bfloat16, device=device)
