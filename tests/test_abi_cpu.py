@@ -101,3 +101,17 @@ def test_defaults_match_the_pages_settings_table(lib):
     # the schedule's end points (the oracle returns T in float32, the precision the kernel takes)
     assert abs(stage.temperature(1, 48) - want["t_start"]) <= 1e-7
     assert abs(stage.temperature(48, 48) - want["t_end"]) <= 1e-7
+
+
+@pytest.mark.parametrize("lang,std", [("c", "c99"), ("c++", "c++17")])
+def test_header_compiles_standalone(lang, std):
+    """include/dg.h is a plain C header: it compiles on its own as C99 and as C++ with warnings on."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    src = f'#include "{HEADER}"\nint main(void) {{ dg_params p; (void)p; return 0; }}\n'
+    out = subprocess.run([cc, f"-std={std}", "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-x", lang, "-"],
+                         input=src, capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
