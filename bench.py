@@ -421,6 +421,16 @@ def run_gpu(args):
         # one-time head preparation: E4M3 codes on the GPU, and their exact bf16 decoding as E
         W, w_exp = dg.quantize_head_e4m3(W)
         E = (W.view(torch.float8_e4m3fn).to(torch.float32) * (2.0 ** w_exp)).to(torch.bfloat16)
+    head_layout = 0
+    if not LOGITS_FP8:
+        # one-time weight preparation, outside every timed region: the bf16 head (and a separate
+        # embedding) re-ordered tile-major, so each operand box of the fused pass is one
+        # contiguous block (bit-identical results; ~1 % faster, measured)
+        W_t = dg.tile_head(W)
+        E = W_t if E is W else dg.tile_head(E)
+        W = W_t
+        head_layout = 1
+        torch.cuda.synchronize()
     h_host = synth.gaussian_hidden(N_POS, D, seed=42)
     if world > 1:
         tdist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
@@ -429,7 +439,8 @@ def run_gpu(args):
     # vocabulary split: every rank works on the same canvases over its rows of the head
     c0 = 0 if split else shard_canvases(world * CANVASES, rank, world)[0]
     p = dg.params(CANVASES, V, D, accept_mode=ACCEPT_MODE, accept_rule=ACCEPT_RULE,
-                  tied=0 if (UNTIED or LOGITS_FP8) else 1, logits_format=1 if LOGITS_FP8 else 0, w_scale_exp=w_exp)
+                  tied=0 if (UNTIED or LOGITS_FP8) else 1, logits_format=1 if LOGITS_FP8 else 0, w_scale_exp=w_exp,
+                  head_layout=head_layout)
     bufs = dg.StepBuffers(p, dev)
     seeds = torch.arange(c0, c0 + CANVASES, dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream()
@@ -574,6 +585,7 @@ def run_gpu(args):
                        "parallelism": (f"vocabulary split x{world} (all-gather of shard partials)" if split else
                                        f"replicas x{world}" if world > 1 else "single GPU"),
                        "l2": "inputs larger than L2 (W/E 1.48 GB streamed per step)",
+                       "head_layout": "tile-major" if head_layout else "row-major",
                        "group": dg.plan(p)["group"], "n_groups": dg.plan(p)["n_groups"]},
             "steps_per_s": 1e3 / ms_per_step,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",

@@ -17,7 +17,8 @@ __all__ = ["DgError", "DgParams", "params", "workspace_size", "plan", "temperatu
            "dg_denoise_step", "dg_stop_check", "dg_stub_hidden", "last_launch_count", "profile_enable",
            "profile_collect", "dg_denoise_stats_noalloc", "dg_debug_set_error", "Workspace", "StepBuffers",
            "decode_batch", "decode_block_ar", "dg_partial_bytes", "dg_denoise_partial", "dg_denoise_merge",
-           "dg_debug_set_counter_wait_limit", "dg_quantize_e4m3", "quantize_head_e4m3", "dg_last_sm_clock"]
+           "dg_debug_set_counter_wait_limit", "dg_quantize_e4m3", "quantize_head_e4m3", "dg_last_sm_clock",
+           "dg_tile_head", "tile_head"]
 
 
 def params(n_canvas, vocab, hidden, **overrides):
@@ -141,6 +142,20 @@ def dg_last_sm_clock(p, ws, stream=None):
     check("dg_last_sm_clock", lib().dg_last_sm_clock(ctypes.byref(p), ws.ptr, ws.nbytes, ctypes.byref(mhz),
                                                      _stream(stream)))
     return float(mhz.value)
+
+
+def dg_tile_head(src, dst, to_rows, stream=None):
+    """Re-order a bf16 [rows, cols] head between row-major (src) and tile-major (dst), or back."""
+    rows, cols = src.shape
+    check("dg_tile_head", lib().dg_tile_head(_ptr(src), _ptr(dst), int(rows), int(cols), int(to_rows),
+                                             _stream(stream)))
+
+
+def tile_head(W, stream=None):
+    """The head in the tile-major layout of params(head_layout=1), as a new [V, d] tensor."""
+    out = torch.empty_like(W)
+    dg_tile_head(W, out, 0, stream)
+    return out
 
 
 def dg_debug_set_counter_wait_limit(ns):

@@ -13,7 +13,7 @@ EXPORTS = ("dg_params_default", "dg_temperature", "dg_workspace_size", "dg_canva
            "dg_stop_check", "dg_stub_hidden", "dg_status_string", "dg_last_launch_count", "dg_plan",
            "dg_profile_enable", "dg_profile_collect", "dg_denoise_stats_noalloc", "dg_debug_set_error",
            "dg_partial_bytes", "dg_denoise_partial", "dg_denoise_merge", "dg_debug_set_counter_wait_limit",
-           "dg_quantize_e4m3", "dg_last_sm_clock")
+           "dg_quantize_e4m3", "dg_last_sm_clock", "dg_tile_head")
 
 
 class DgParams(ctypes.Structure):
@@ -22,7 +22,7 @@ class DgParams(ctypes.Structure):
                 ("t_end", ctypes.c_float), ("eb_bound", ctypes.c_float), ("stop_thresh", ctypes.c_float),
                 ("stability", ctypes.c_int), ("tied", ctypes.c_int), ("group", ctypes.c_int),
                 ("accept_mode", ctypes.c_int), ("accept_rule", ctypes.c_int), ("logits_format", ctypes.c_int),
-                ("w_scale_exp", ctypes.c_int)]
+                ("w_scale_exp", ctypes.c_int), ("head_layout", ctypes.c_int)]
 
 
 class DgError(RuntimeError):
@@ -80,6 +80,8 @@ def lib():
         L.dg_quantize_e4m3.restype = i32
         L.dg_last_sm_clock.argtypes = [P, vp, sz, ctypes.POINTER(ctypes.c_float), vp]
         L.dg_last_sm_clock.restype = i32
+        L.dg_tile_head.argtypes = [vp, vp, ctypes.c_longlong, i32, i32, vp]
+        L.dg_tile_head.restype = i32
         L.dg_profile_enable.argtypes = [i32]
         L.dg_profile_enable.restype = i32
         L.dg_profile_collect.argtypes = [ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_float),

@@ -77,6 +77,7 @@ bool params_ok(const dg_params* p) {
     if (p->accept_mode != 0 && p->accept_mode != 1) return false;
     if (p->accept_rule != 0 && p->accept_rule != 1) return false;
     if (p->logits_format != 0 && p->logits_format != 1) return false;
+    if (p->head_layout != 0 && p->head_layout != 1) return false;
     return true;
 }
 
@@ -109,6 +110,21 @@ bool encode_blocks_3d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t 
     cuuint64_t dims[3] = {64, rows, cols / 64};
     cuuint64_t strides[2] = {cols * 2, 128};
     cuuint32_t box[3] = {64, box_rows, box_blocks};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A bf16 [rows, cols] head in the tile-major layout (tiled_index): {64 columns, 128 rows,
+// (rows/128) (cols/64) atoms}, atoms 16 KB apart, so a box of {64, 128, box_blocks} at atom z
+// is box_blocks consecutive atoms of one row tile - one contiguous block of memory.
+bool encode_tiled_3d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_blocks) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || cols % 64 != 0 || rows % 128 != 0) return false;
+    cuuint64_t dims[3] = {64, 128, (rows / 128) * (cols / 64)};
+    cuuint64_t strides[2] = {128, 128 * 128};
+    cuuint32_t box[3] = {64, 128, box_blocks};
     cuuint32_t es[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -204,6 +220,8 @@ dg_status make_plan(const dg_params* p, int pairs, Plan* pl) {
     }
     q.n_slots = q.n_groups * q.max_seg;
     q.fp8 = p->logits_format == 1;
+    q.tiled = p->head_layout == 1;
+    if (q.fp8 && q.tiled) return DG_EUNSUPPORTED;
     *pl = q;
     return DG_OK;
 }
@@ -249,10 +267,13 @@ dg_status launch_fused_and_combine(const dg_params* p, const Plan& pl, const Lay
     const bool maps_ok =
         pl.fp8 ? encode_bytes_3d(&fa.map_h, at<void>(ws, L.hq), pl.N, pl.d, kTileM, 2) &&
                      encode_bytes_3d(&fa.map_w, io.W, io.vocab_rows, pl.d, kBV / 2, 2)
-               : encode_blocks_3d(&fa.map_h, io.h, pl.N, pl.d, kTileM, kKChunk / 64) &&
-                     encode_blocks_3d(&fa.map_w, io.W, io.vocab_rows, pl.d, kBV / 2, kKChunk / 64);
-    if (!maps_ok ||
-        !encode_blocks_3d(&fa.map_e, io.E, io.vocab_rows, pl.d, kVChunk, pl.slice / 128) ||
+        : pl.tiled ? encode_blocks_3d(&fa.map_h, io.h, pl.N, pl.d, kTileM, kKChunk / 64) &&
+                         encode_tiled_3d(&fa.map_w, io.W, io.vocab_rows, pl.d, kKChunk / 64) &&
+                         encode_tiled_3d(&fa.map_e, io.E, io.vocab_rows, pl.d, pl.slice / 128)
+                   : encode_blocks_3d(&fa.map_h, io.h, pl.N, pl.d, kTileM, kKChunk / 64) &&
+                         encode_blocks_3d(&fa.map_w, io.W, io.vocab_rows, pl.d, kBV / 2, kKChunk / 64) &&
+                         encode_blocks_3d(&fa.map_e, io.E, io.vocab_rows, pl.d, kVChunk, pl.slice / 128);
+    if (!maps_ok || (pl.fp8 && !encode_blocks_3d(&fa.map_e, io.E, io.vocab_rows, pl.d, kVChunk, pl.slice / 128)) ||
         !encode_blocks_3d(&fa.map_p, at<void>(ws, L.pbuf), prow_total, kCanvas, kVChunk, 2))
         return DG_ECUDA;
     int32_t* stop = at<int32_t>(ws, L.stop);
@@ -274,6 +295,7 @@ dg_status launch_fused_and_combine(const dg_params* p, const Plan& pl, const Lay
     fa.vocab_offset = io.vocab_offset;
     fa.d = pl.d;
     fa.G = pl.group;
+    fa.tiled = pl.tiled;
     fa.keep_w_stages = (io.E == io.W && !pl.fp8) ? (pl.d / kKChunk) * kKeepWTenths / 10 : 0;
     if (pl.fp8) {
         fa.row_exp = at<int32_t>(ws, L.hexp);
@@ -611,6 +633,25 @@ dg_status dg_quantize_e4m3(const void* src_dev, long long rows, int cols, int pe
     return DG_OK;
 }
 
+dg_status dg_tile_head(const void* src_dev, void* dst_dev, long long rows, int cols, int to_rows, void* stream) {
+    g_last_launches = 0;
+    if (!src_dev || !dst_dev || rows < 128 || rows % 128 != 0 || cols < 64 || cols % 64 != 0) return DG_EINVAL;
+    if (to_rows != 0 && to_rows != 1) return DG_EINVAL;
+    if (!aligned16(src_dev) || !aligned16(dst_dev)) return DG_EINVAL;
+    const uintptr_t bytes = static_cast<uintptr_t>(rows) * static_cast<uintptr_t>(cols) * 2;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(src_dev), b = reinterpret_cast<uintptr_t>(dst_dev);
+    if (a < b + bytes && b < a + bytes) return DG_EINVAL;
+    const long long work = rows * (cols / 8);
+    long long blocks = (work + 255) / 256;
+    const long long cap = static_cast<long long>(device_sm_count()) * 16;
+    if (cap > 0 && blocks > cap) blocks = cap;
+    dg_tile_head_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16*>(src_dev), static_cast<__nv_bfloat16*>(dst_dev), rows, cols, to_rows);
+    if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
+    g_last_launches = 1;
+    return DG_OK;
+}
+
 dg_status dg_debug_set_counter_wait_limit(unsigned long long ns) {
     g_counter_wait_ns = ns == 0 ? DG_WAIT_LIMIT_NS : ns;
     return DG_OK;
@@ -743,7 +784,7 @@ dg_status dg_stub_hidden(const dg_params* p, int step, float gain, float noise, 
     if (cap > 0 && blocks > cap) blocks = cap;
     dg_stub_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(
         seeds_dev, static_cast<const __nv_bfloat16*>(E_dev), tokens_dev, at<int32_t>(workspace_dev, L.stop),
-        static_cast<__nv_bfloat16*>(h_dev), a_s, gain, noise, step, pl.d, pl.V, pl.N);
+        static_cast<__nv_bfloat16*>(h_dev), a_s, gain, noise, step, pl.d, pl.V, pl.N, pl.tiled);
     if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
     g_last_launches = 1;
     return DG_OK;

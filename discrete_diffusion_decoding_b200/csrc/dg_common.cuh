@@ -77,6 +77,13 @@ enum : uint32_t { kTagInit = 0, kTagRenoise = 1, kTagStubTarget = 2, kTagStubNoi
 // sampled acceptance: counter (v / 64, step, canvas, kTagSample + 256 i), one per 64-entry chunk
 constexpr uint32_t kTagSample = 4;
 
+// ------------------------------------------------------------------ tile-major head layout
+// Element (v, c) of a [V, d] head stored tile-major: atoms of 128 rows x 64 columns, ordered
+// by row tile then column atom, each atom row-major (64 contiguous columns per row).
+__host__ __device__ inline size_t tiled_index(long long v, int c, int d) {
+    return (static_cast<size_t>(v >> 7) * (d >> 6) + (c >> 6)) * 8192 + static_cast<size_t>(v & 127) * 64 + (c & 63);
+}
+
 // ------------------------------------------------------------------ plan and layout
 struct Plan {
     int C, N, V, d;
@@ -87,6 +94,7 @@ struct Plan {
     int max_seg;      // partial slots per group
     int n_slots;      // n_groups * max_seg
     int fp8;          // E4M3 logits operands (the workspace then holds the quantised hidden states)
+    int tiled;        // W and E in the tile-major head layout (tiled_index)
 };
 
 struct Layout {

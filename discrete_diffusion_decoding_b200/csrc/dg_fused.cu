@@ -329,9 +329,13 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                         } else {
                             arm(slot, e_box_bytes);
                             // this CTA's half of the column slice (n_ech atoms of 64 columns) in one 3-D box
-                            tma_load_3d_pair_hint(st, &a.map_e, full_leader(slot), 0,
-                                                  vocab0(t, q) + vc * kVChunk,
-                                                  (d0 + static_cast<int>(prank) * (a.slice / 2)) / 64, pol_stream);
+                            const int er = vocab0(t, q) + vc * kVChunk;
+                            const int ec = (d0 + static_cast<int>(prank) * (a.slice / 2)) / 64;
+                            if (a.tiled)      // tile (er / 128, ec): n_ech consecutive atoms, one contiguous block
+                                tma_load_3d_pair_hint(st, &a.map_e, full_leader(slot), 0, 0,
+                                                      (er >> 7) * (a.d >> 6) + ec, pol_stream);
+                            else
+                                tma_load_3d_pair_hint(st, &a.map_e, full_leader(slot), 0, er, ec, pol_stream);
                         }
                     }
                 }
@@ -353,11 +357,14 @@ __device__ __forceinline__ void fused_pass(const FusedArgs& a) {
                             if (a_side) {
                                 tma_load_3d_pair(st, &a.map_h, full_leader(slot), 0, row0, kc * (kKChunk / 64));
                             } else {
+                                // row-major: box at rows v0, column block kc * 2; tiled: the two atoms of
+                                // tile (v0 / 128, kc * 2), one contiguous 32 KB block
+                                const int wy = a.tiled ? 0 : v0;
+                                const int wz = a.tiled ? (v0 >> 7) * (a.d >> 6) + kc * 2 : kc * (kKChunk / 64);
                                 if (kc < a.keep_w_stages)
-                                    tma_load_3d_pair(st, &a.map_w, full_leader(slot), 0, v0, kc * (kKChunk / 64));
+                                    tma_load_3d_pair(st, &a.map_w, full_leader(slot), 0, wy, wz);
                                 else
-                                    tma_load_3d_pair_hint(st, &a.map_w, full_leader(slot), 0, v0,
-                                                          kc * (kKChunk / 64), pol_stream);
+                                    tma_load_3d_pair_hint(st, &a.map_w, full_leader(slot), 0, wy, wz, pol_stream);
                             }
                         }
                     }

@@ -33,6 +33,8 @@ struct FusedArgs {
     int C, V, d, G, slice, n_groups, steps_per_tile, max_seg;
     int vocab_offset;    // vocabulary index of row 0 of W / E (a shard of the vocabulary; 0 otherwise):
                          // added to the argmax and sample indices and to the sampled mode's chunk counter
+    int tiled;           // W and E in the tile-major head layout (dg_tile_head): atoms of 128 rows x 64
+                         // columns, [row tile][column atom], so every 3-D box is one contiguous block
     int keep_w_stages;   // E aliases W: the first keep_w_stages hidden-column stages of every W
                          // tile keep normal L2 priority, so the self-conditioning pass finds them
                          // there (0 when E is a separate matrix)
@@ -133,6 +135,8 @@ __global__ void dg_stop_kernel(const float* entropy, const int32_t* argmax, int3
                                int32_t* stop, float stop_thresh, int stability, int step, GroupAcceptArgs ga);
 __global__ void dg_stub_kernel(const uint64_t* seeds, const __nv_bfloat16* E, const int32_t* tokens,
                                const int32_t* stop, __nv_bfloat16* h, float a_s, float gain, float noise, int step,
-                               int d, int V, int N);
+                               int d, int V, int N, int tiled);
+// Row-major [V, d] bf16 head -> tile-major (or back when to_rows is 1).
+__global__ void dg_tile_head_kernel(const __nv_bfloat16* src, __nv_bfloat16* dst, long long V, int d, int to_rows);
 
 }  // namespace dg

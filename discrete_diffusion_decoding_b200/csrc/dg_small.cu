@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(256) dg_stop_kernel(const float* entropy, cons
 // (w2, w3) give 4j+2, 4j+3 with u1 = (w+1) 2^-32 and u2 = w' 2^-32.
 __global__ void dg_stub_kernel(const uint64_t* seeds, const __nv_bfloat16* E, const int32_t* tokens,
                                const int32_t* stop, __nv_bfloat16* h, float a_s, float gain, float noise, int step,
-                               int d, int V, int N) {
+                               int d, int V, int N, int tiled) {
     const int q = d / 4;
     const long long total = static_cast<long long>(N) * q;
     for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
@@ -148,8 +148,11 @@ __global__ void dg_stub_kernel(const uint64_t* seeds, const __nv_bfloat16* E, co
             nz[2 * p] = rad * cs;
             nz[2 * p + 1] = rad * sn;
         }
-        const uint2 et = *reinterpret_cast<const uint2*>(E + static_cast<size_t>(tgt) * d + 4 * j);
-        const uint2 ex = *reinterpret_cast<const uint2*>(E + static_cast<size_t>(x) * d + 4 * j);
+        // four consecutive columns of a row: contiguous in either head layout
+        const size_t ot = tiled ? tiled_index(tgt, 4 * j, d) : static_cast<size_t>(tgt) * d + 4 * j;
+        const size_t ox = tiled ? tiled_index(x, 4 * j, d) : static_cast<size_t>(x) * d + 4 * j;
+        const uint2 et = *reinterpret_cast<const uint2*>(E + ot);
+        const uint2 ex = *reinterpret_cast<const uint2*>(E + ox);
         const __nv_bfloat162* bt = reinterpret_cast<const __nv_bfloat162*>(&et);
         const __nv_bfloat162* bx = reinterpret_cast<const __nv_bfloat162*>(&ex);
         float vt[4] = {__low2float(bt[0]), __high2float(bt[0]), __low2float(bt[1]), __high2float(bt[1])};
@@ -163,6 +166,22 @@ __global__ void dg_stub_kernel(const uint64_t* seeds, const __nv_bfloat16* E, co
         pk.x = *reinterpret_cast<uint32_t*>(&o0);
         pk.y = *reinterpret_cast<uint32_t*>(&o1);
         *reinterpret_cast<uint2*>(h + static_cast<size_t>(n) * d + 4 * j) = pk;
+    }
+}
+
+// Row-major <-> tile-major head (tiled_index): one thread per 8 consecutive columns of a row
+// (16 bytes, inside one 64-column atom in both layouts).
+__global__ void dg_tile_head_kernel(const __nv_bfloat16* src, __nv_bfloat16* dst, long long V, int d, int to_rows) {
+    const int per_row = d / 8;
+    const long long total = V * per_row;
+    for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
+         e += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long v = e / per_row;
+        const int c = static_cast<int>(e % per_row) * 8;
+        const size_t rm = static_cast<size_t>(v) * d + c;
+        const size_t tl = tiled_index(v, c, d);
+        const uint4 x = *reinterpret_cast<const uint4*>(src + (to_rows ? tl : rm));
+        *reinterpret_cast<uint4*>(dst + (to_rows ? rm : tl)) = x;
     }
 }
 

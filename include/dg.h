@@ -122,6 +122,18 @@ typedef struct {
                          *   The pages cite quantised deployments of the model (axbrief.com brief,
                          *   GGUF sizes) but define no quantisation of this stage. */
     int w_scale_exp;    /* logits_format 1: the power-of-two exponent of the head's scale */
+    int head_layout;    /* storage order of the bf16 head W_dev and embedding E_dev:
+                         *   0 = row-major [V, d] (default);
+                         *   1 = tile-major, from dg_tile_head: atoms of 128 vocabulary rows x
+                         *       64 hidden columns, ordered by row tile then column atom, each
+                         *       atom row-major - element (v, c) at
+                         *       ((v / 128) (d / 64) + c / 64) 8192 + (v % 128) 64 + c % 64.
+                         *       Every operand tile of the fused kernel is then one contiguous
+                         *       block of memory instead of 128 rows of 128 or 256 bytes.  The
+                         *       results are bit-identical to those of layout 0.  Row v0 (a
+                         *       multiple of 128) still starts at element v0 d, so a vocabulary
+                         *       shard is the same sub-array in both layouts.  Not with
+                         *       logits_format 1 (DG_EUNSUPPORTED). */
 } dg_params;
 
 /* Fill a dg_params with the pages' defaults for C canvases of a (V, d) head. */
@@ -323,6 +335,16 @@ dg_status dg_denoise_merge(const dg_params* p, int step, int n_parts, const void
                            const uint64_t* seeds_dev, int32_t* tokens_dev, float* entropy_dev, int32_t* argmax_dev,
                            uint8_t* accept_dev, float* lse_dev, float* selfcond_dev, void* workspace_dev,
                            size_t workspace_bytes, void* stream);
+
+/*
+ * Re-order a bf16 [rows, cols] head between row-major and the tile-major layout of
+ * dg_params.head_layout 1: to_rows 0 writes tile-major dst_dev from row-major src_dev,
+ * to_rows 1 the reverse.  rows a multiple of 128, cols a multiple of 64, both pointers
+ * 16-byte aligned and not overlapping (DG_EINVAL otherwise); rows * cols elements each,
+ * owned by the caller.  One launch, asynchronous on `stream`.  A one-time conversion of the
+ * weights, not a step of the decode.
+ */
+dg_status dg_tile_head(const void* src_dev, void* dst_dev, long long rows, int cols, int to_rows, void* stream);
 
 /*
  * E4M3 quantisation (the 8-bit format of logits_format 1): sign bit, 4 exponent bits with

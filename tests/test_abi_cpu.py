@@ -115,3 +115,19 @@ def test_header_compiles_standalone(lang, std):
     out = subprocess.run([cc, f"-std={std}", "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-x", lang, "-"],
                          input=src, capture_output=True, text=True, timeout=60)
     assert out.returncode == 0, out.stderr
+
+
+
+def test_tile_head_argument_checks_without_device(lib):
+    """dg_tile_head refuses bad shapes, null and overlapping pointers before touching a device."""
+    lib.dg_tile_head.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int, ctypes.c_int,
+                                 ctypes.c_void_p]
+    lib.dg_tile_head.restype = ctypes.c_int
+    a, b = 1 << 20, 1 << 30                      # never dereferenced: every call below fails its checks
+    for args in ((None, b, 256, 128, 0), (a, None, 256, 128, 0), (a, b, 200, 128, 0), (a, b, 256, 96, 0),
+                 (a, b, 0, 128, 0), (a, b, 256, 128, 2), (a + 8, b, 256, 128, 0), (a, a + 4096, 256, 128, 0)):
+        assert lib.dg_tile_head(*args, None) == -1, args
+    from discrete_diffusion_decoding_b200 import _abi
+    p = _abi.DgParams()
+    lib.dg_params_default(ctypes.byref(p), 1, 4096, 512)
+    assert p.head_layout == 0
