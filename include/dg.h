@@ -227,7 +227,8 @@ dg_status dg_debug_set_error(const dg_params* p, void* workspace_dev, size_t wor
  * of 2 s; 0 restores 2 s.  A wait that runs out makes the kernel leave early and record
  * the error word exactly as a stalled peer would (DG_ETIMEOUT from dg_stop_check, poisoned
  * results).  The waits that drain a CTA's own loads and tensor-core operations keep their
- * 2 s limit, so none is in flight when a CTA leaves.  Always returns DG_OK.
+ * 2 s limit (they wait for the CTA's own loads to land), so none is in flight when a CTA
+ * leaves.  Always returns DG_OK.
  */
 dg_status dg_debug_set_counter_wait_limit(unsigned long long ns);
 
@@ -236,7 +237,8 @@ dg_status dg_debug_set_counter_wait_limit(unsigned long long ns);
  *   h_i = gain * (a E[tgt_i] + (1 - a) E[x_i]) + noise * n_i,   a = s / max_steps,
  * tgt_i uniform over V (Philox tag 2, step 0), n_i standard normal by Box-Muller on
  * Philox tag 3 words (counter (i*d/4 + k/4, s, c, 3)).  Computed in fp32, stored bf16.
- * Only canvases not yet stopped are written (the workspace holds the flags).
+ * E_dev is read in the layout p->head_layout names.  Only canvases not yet stopped are
+ * written (the workspace holds the flags).
  */
 dg_status dg_stub_hidden(const dg_params* p, int step, float gain, float noise, const uint64_t* seeds_dev,
                          const void* E_dev, const int32_t* tokens_dev, void* h_dev, void* workspace_dev,
