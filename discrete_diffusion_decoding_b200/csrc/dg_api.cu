@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "../../include/dg.h"
@@ -251,6 +252,24 @@ PartialLayout partial_layout(int N, int d) {
     return P;
 }
 
+// Launch a kernel that consumes only what the kernel before it on the stream wrote, with
+// programmatic stream serialization: it is set up while its predecessor runs and waits
+// (griddepcontrol.wait at its top) for the predecessor to complete, hiding the launch gap.
+template <class... KArgs, class... Args>
+cudaError_t launch_after(void (*kern)(KArgs...), dim3 grid, dim3 block, cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 dg_status launch_fused_and_combine(const dg_params* p, const Plan& pl, const Layout& L, void* ws, int step,
                                    const PassIO& io, cudaStream_t s) {
     if (!fused_attr_set()) return DG_ECUDA;
@@ -369,8 +388,7 @@ dg_status launch_fused_and_combine(const dg_params* p, const Plan& pl, const Lay
     ca.bound = p->eb_bound;
     ca.step = step;
     ca.V = pl.V;
-    dg_combine_kernel<<<combine_grid(pl.N, pl.d), 256, 0, s>>>(ca);
-    if (cudaGetLastError() != cudaSuccess) return DG_ECUDA;
+    if (launch_after(dg_combine_kernel, combine_grid(pl.N, pl.d), dim3(256), s, ca) != cudaSuccess) return DG_ECUDA;
     return DG_OK;
 }
 
@@ -386,10 +404,10 @@ dg_status launch_stop(const dg_params* p, const Plan& pl, const Layout& L, void*
                       const int32_t* argmax_dev, uint8_t* accept_dev, cudaStream_t s) {
     GroupAcceptArgs ga{p->accept_rule, p->eb_bound, at<int32_t>(ws, L.kept), seeds_dev, tokens_dev, accept_dev,
                        pl.V};
-    dg_stop_kernel<<<pl.C, kCanvas, 0, s>>>(entropy_dev, argmax_dev, at<int32_t>(ws, L.prev_argmax),
-                                            at<int32_t>(ws, L.stable), at<int32_t>(ws, L.stop), p->stop_thresh,
-                                            p->stability, step, ga);
-    return cudaGetLastError() == cudaSuccess ? DG_OK : DG_ECUDA;
+    const cudaError_t e = launch_after(dg_stop_kernel, dim3(pl.C), dim3(kCanvas), s, entropy_dev, argmax_dev,
+                                       at<int32_t>(ws, L.prev_argmax), at<int32_t>(ws, L.stable),
+                                       at<int32_t>(ws, L.stop), p->stop_thresh, p->stability, step, ga);
+    return e == cudaSuccess ? DG_OK : DG_ECUDA;
 }
 
 }  // namespace

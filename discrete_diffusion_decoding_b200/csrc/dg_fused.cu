@@ -797,6 +797,7 @@ __device__ void finish_position(const Finish& f, int n, int c, int crow, float M
 // the unnormalised numerator sum_s 2^(m_s-M) O_s instead.  CTA (0, 0) also clears
 // the fused kernel's group counters for its next launch.
 __global__ void __launch_bounds__(256) dg_combine_kernel(const CombineArgs a) {
+    griddep_wait();                         // launched after the fused pass it merges
     __shared__ float sh_w[kMaxSlotsPerTile];
     __shared__ int sh_slot[kMaxSlotsPerTile];
     __shared__ int n_slots_s;

@@ -118,6 +118,10 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
     return ok != 0;
 }
 
+// Wait until the grids this one depends on (launched before it on the stream) have
+// completed and their memory is visible; a no-op for a normally launched grid.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Transaction bytes counted on a local barrier without a copy: stands in for bytes that
 // were expected but will never be sent (the drain of an aborted pass).
 __device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {

@@ -91,6 +91,8 @@ __device__ void group_accept(const float* entropy, const GroupAcceptArgs& ga, in
 __global__ void __launch_bounds__(256) dg_stop_kernel(const float* entropy, const int32_t* argmax,
                                                       int32_t* prev_argmax, int32_t* stable, int32_t* stop,
                                                       float stop_thresh, int stability, int step, GroupAcceptArgs ga) {
+    // launched after the kernel that wrote this step's entropy and argmax: wait for it
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int c = blockIdx.x;
     if (stop[c]) return;
     if (ga.rule == 1 && ga.tokens != nullptr) group_accept(entropy, ga, c, step);
